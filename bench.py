@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Throughput of the B200 MoE FFN layer (tokens/s) with its roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+    python bench.py --impl reference ...     # the CPU oracle as the reference arm
+
+One step = one forward of the whole layer (router GEMM, selection, dispatch,
+gate/up GEMM + SwiGLU, down GEMM x weight, combine) over one batch of seeded
+synthetic tokens, with every input already resident in HBM.  Under torchrun
+each rank runs an independent replica (tokens are independent: no collective
+on the data path); the timed region is bracketed by a barrier and device
+synchronisation, and the max over ranks is reported.  The JSON line also
+carries the roofline of the dominant kernel, the oracle's CPU throughput, an
+end-to-end figure through the C ABI with host buffers, and SM clocks sampled
+during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and % roofline (HBM GB/s decode, TFLOP/s prefill), 1×B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU work of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- work model
+
+def layer_work(wl, touched: int):
+    """Algorithmic FLOPs and HBM bytes of one layer call and of the gate/up
+    GEMM (the dominant kernel)."""
+    T, H, E, k, I, Is = wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is
+    el = 2  # bf16
+    flops = T * (2 * k * 3 * H * I + 2 * 3 * H * Is + 2 * H * E)
+    bytes_ = (touched * 3 * H * I + 3 * H * Is + E * H + 2 * T * H) * el
+    g1_flops = 2 * T * k * 2 * I * H + 2 * T * 2 * Is * H
+    g1_bytes = (touched * 2 * I * H + 2 * Is * H      # weights streamed
+                + T * k * H + T * H                   # gathered + shared activations
+                + T * k * I + T * Is) * el            # SwiGLU outputs
+    return {"flops": flops, "bytes": bytes_, "g1_flops": g1_flops, "g1_bytes": g1_bytes}
+
+
+# ---------------------------------------------------------------- our arm
+
+def cfg_of(B, wl):
+    return B.MoeConfig(T=wl.T, H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
+                       n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
+                       norm_topk_prob=wl.norm_topk_prob,
+                       routed_scaling_factor=wl.routed_scaling_factor)
+
+
+def launches_per_step(B, cfg):
+    from sigmoid_top_routing_warp_b200 import build as _b  # noqa: F401
+    permute = 1 if cfg.T * cfg.k <= 4096 else 3
+    # router GEMM, selection, permute, gather, gate/up GEMM, down GEMM, combine
+    return 2 + permute + 1 + 2 + 1
+
+
+def run_ours(args, world, rank, local):
+    from sigmoid_top_routing_warp_b200 import binding as B
+    from sigmoid_top_routing_warp_b200 import workloads as W
+
+    wl = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    inp = W.make_inputs(wl, device=dev, seed=wl.seed + rank)
+    cfg = cfg_of(B, wl)
+    ws = B.alloc_workspace(cfg, device=dev)
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                      inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    B.moe_check_device_status(ws)
+    offs = B.ws_view(ws, cfg, "offsets").cpu().numpy()
+    touched = int((np.diff(offs) > 0).sum())
+
+    # timed region: K steps, stage events recorded on the launching stream
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_NUM_STAGES + 1)]
+           for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)  # materialise the handles
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    with ClockSampler(dev.index) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    B.moe_check_device_status(ws)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(world, ms)
+    stages = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(B.MOE_NUM_STAGES)]
+                       for i in range(K)])
+    stage_ms = stages.mean(0)
+
+    # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        B.moe_forward(cfg, x_dev, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                      inp["w13s"], inp["w2s"], out, ws, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
+    barrier(world)
+    return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
+            "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
+            "launches": launches_per_step(B, cfg) * K, "B": B}
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(wl, inp, seconds: float):
+    """Time the CPU oracle (router logits, selection and layer) on a bounded
+    sample of the workload's tokens; returns (tokens/s, threads, sample)."""
+    from oracle import oracle as O
+
+    def u16(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    threads = O.set_threads(os.cpu_count() or 1)
+    wg = u16(inp["w_router"])
+    bias = inp["bias"].cpu().numpy()
+    w13s, w2s = u16(inp["w13s"]), u16(inp["w2s"])
+    n = max(1, min(wl.T, threads))
+    spent, done, rounds = 0.0, 0, 0
+    rng = np.random.default_rng(1)
+    while spent < seconds and rounds < 6:
+        toks = rng.choice(wl.T, size=min(n, wl.T), replace=False)
+        x = u16(inp["x"][torch.as_tensor(toks, device=inp["x"].device)])
+        oc = O.Config(T=len(toks), H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
+                      n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
+                      norm_topk_prob=wl.norm_topk_prob,
+                      routed_scaling_factor=wl.routed_scaling_factor)
+        # routing needs only W_g; the layer needs the experts these tokens use
+        t0 = time.perf_counter()
+        L = O.router_logits(oc, x, wg).astype(np.float32)
+        idx, w, _ = O.route(oc, L, bias)
+        t_route = time.perf_counter() - t0
+        used = np.unique(idx)
+        sel = torch.as_tensor(used, device=inp["w13"].device)
+        w13, w2 = u16(inp["w13"][sel]), u16(inp["w2"][sel])
+        remap = np.full(wl.E, -1, np.int64)
+        remap[used] = np.arange(used.size)
+        oc2 = O.Config(**{**oc.__dict__, "E": int(used.size)})
+        t1 = time.perf_counter()
+        O.layer(oc2, x, remap[idx].astype(np.int32), w, w13, w2, w13s, w2s)
+        spent += t_route + time.perf_counter() - t1
+        done += len(toks)
+        rounds += 1
+        n = min(wl.T, n * 2)
+    return done / spent, threads, "%d tokens of workload %s (%d rounds, %.1f s)" % (
+        done, wl.name, rounds, spent)
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle as it stands, on this host's cores."""
+    if rank != 0:
+        return None
+    from sigmoid_top_routing_warp_b200 import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(wl, device=dev)
+    per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    rates = []
+    for i in range(args.warmup + args.steps):
+        r, threads, sample = oracle_sample(wl, inp, per_step)
+        if i >= args.warmup:
+            rates.append(r)
+    value = float(statistics.median(rates))
+    ms = wl.T / value * 1e3
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+                       "I": wl.I, "n_shared": wl.n_shared},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    peaks, peak_src = load_peaks()
+    r = run_ours(args, world, rank, local)
+    wl, K = r["wl"], args.steps
+    work = layer_work(wl, r["touched"])
+    value = world * wl.T * K / (r["ms"] / 1e3)
+    stage_names = r["B"].STAGE_NAMES
+    g1_ms = float(r["stage_ms"][3])
+    hbm_bound = work["bytes"] / (peaks["hbm_gbs"] * 1e9) >= work["flops"] / (
+        peaks["bf16_tflops"] * 1e12)
+    if hbm_bound:
+        ach = work["g1_bytes"] / (g1_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": None}
+    else:
+        ach = work["g1_flops"] / (g1_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None}
+    roof.update({"kernel": "grouped_gemm_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
+                 "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
+                 "launch_ms": g1_ms, "peak_source": peak_src})
+    layer_ms = r["ms"] / K
+    layer = {"ms": layer_ms,
+             "hbm_gbs": work["bytes"] / (layer_ms / 1e3) / 1e9,
+             "tflops": work["flops"] / (layer_ms / 1e3) / 1e12,
+             "t_roof_ms": 1e3 * max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                                    work["flops"] / (peaks["bf16_tflops"] * 1e12))}
+    layer["frac_of_roofline"] = layer["t_roof_ms"] / layer_ms
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": layer_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+                       "I": wl.I, "n_shared": wl.n_shared, "n_group": wl.n_group,
+                       "topk_group": wl.topk_group, "experts_touched": r["touched"],
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
+                             % (work["bytes"] / 1e9)},
+            "roofline": roof, "layer_roofline": layer,
+            "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
+            "gpu_launches": r["launches"], "clocks": r["clocks"],
+            "e2e": {"value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, sample = oracle_sample(wl, r["inp"], args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

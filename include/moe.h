@@ -1,0 +1,202 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE FFN layer library
+ *          (libmoe_b200.so, built from sigmoid_top_routing_warp_b200/csrc).
+ *
+ * The layer is the dots-style fine-grained mixture-of-experts feed-forward
+ * block.  Per token x (a row of H values) it computes
+ *
+ *   logits  L = x W_g^T                        (router, E experts)
+ *   scores  s = sigmoid(L)
+ *   choice  c = s + b  (b: per-expert bias, used only for choosing; optional
+ *           group limit: keep the topk_group groups of E/n_group contiguous
+ *           experts with the largest sum of their group_topn best keys)
+ *   idx     = the k experts with the largest c (ties: lower expert first),
+ *             listed in that order ("slot" order)
+ *   w_j     = s[idx_j] / sum_j s[idx_j] (if norm_topk_prob) * rsf
+ *   out     = SwiGLU_shared(x) + sum_j w_j * SwiGLU_{idx_j}(x)
+ *   SwiGLU_e(x) = W2_e ( SiLU(W_gate,e x) * (W_up,e x) )
+ *
+ * Sources (web pages, cited by title and section):
+ *   "dots3-note 架构深度解析：16B 激活参数的 280B MoE 如何实现高效推理" (mlqm.cn),
+ *     section 稀疏激活：Top-8 路由: sigmoid scoring, noaux_tc routing,
+ *     norm_topk_prob, 256 routed + 1 shared experts, top-8, hidden 5120,
+ *     moe_intermediate_size 1536, BF16 / FP8 weights.
+ *   "Xiaohongshu dots3 note Open Source Deep Dive: 280B MoE Multimodal Model"
+ *     (happyrock.cloud), §3.1 Expert Routing Mechanism (gate, top-k,
+ *     renormalise, shared + weighted routed sum), §3.3 layer diagram,
+ *     §8.2 Ascend Adaptation Architecture (FUSED_MC2:
+ *     dispatch -> gmm1 -> swiglu -> gmm2 -> combine).
+ *   "🤗 Transformers 中的 dots.llm1（Dots1）模型" (blog.gitcode.com), table
+ *     MoE 路由与专家相关字段 (n_group, topk_group, norm_topk_prob,
+ *     routed_scaling_factor, moe_intermediate_size) and the parallel-plan
+ *     paragraph (packed gate_up_proj, grouped_gemm experts).
+ *
+ * Conventions for every entry point:
+ *   - Every data pointer is DEVICE memory owned by the caller.  The library
+ *     never allocates, frees or keeps a pointer after the call returns.
+ *   - Matrices are row-major and densely packed.  bf16 values are stored as
+ *     IEEE bfloat16 (2 bytes); fp32 as IEEE binary32.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) on the current CUDA device.  No call
+ *     synchronises with the host except moe_check_device_status.
+ *   - Argument and shape errors are detected on the host before anything is
+ *     launched: the call returns a non-zero moe_status_t and
+ *     moe_get_last_error() describes it.  Nothing is written in that case.
+ *   - Errors the kernels detect (a bounded wait that ran out) are recorded in
+ *     a status word inside the workspace; read it with
+ *     moe_check_device_status.
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, bad shape or option            */
+    MOE_ERR_UNSUPPORTED = 2, /* valid layer the kernels do not handle         */
+    MOE_ERR_WORKSPACE = 3,   /* workspace smaller than moe_workspace_size()  */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed            */
+    MOE_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out           */
+} moe_status_t;
+
+typedef enum {
+    MOE_DTYPE_BF16 = 0 /* bf16 activations and weights, fp32 accumulation */
+} moe_dtype_t;
+
+/* Layer description.  Field names follow the Dots1 / DeepSeek-V3 config:
+ *   T                      tokens in this call (rows of x), >= 0
+ *   H                      hidden size (multiple of 128)
+ *   E                      routed experts (n_routed_experts), 1..1024
+ *   k                      experts per token (num_experts_per_tok), 1..min(E, 32)
+ *   I                      expert intermediate size (moe_intermediate_size),
+ *                          multiple of 128
+ *   n_shared               shared experts (n_shared_experts) >= 0; they act as
+ *                          one SwiGLU of width n_shared * I
+ *   n_group, topk_group    group-limited choice (1, 1 = plain top-k)
+ *   group_topn             keys summed into a group score (2)
+ *   norm_topk_prob         non-zero: divide weights by their sum
+ *   routed_scaling_factor  multiplies the routed weights (1.0)
+ *   dtype                  moe_dtype_t
+ *   flags                  0 (reserved)                                     */
+typedef struct {
+    int32_t T, H, E, k, I, n_shared;
+    int32_t n_group, topk_group, group_topn;
+    int32_t norm_topk_prob;
+    float routed_scaling_factor;
+    int32_t dtype;
+    uint32_t flags;
+} moe_config_t;
+
+/* A cudaStream_t. */
+typedef void* moe_stream_t;
+
+/* Number of stage events moe_forward records when given an event array:
+ * event i is recorded when stage i starts, the last one after the last
+ * stage.  Stages: 0 router GEMM, 1 router selection, 2 dispatch (histogram,
+ * scan, scatter, gather), 3 gate/up GEMM + SwiGLU, 4 down GEMM x weight,
+ * 5 combine. */
+#define MOE_NUM_STAGES 6
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* moe_get_last_error(void);
+
+/* Bytes of device workspace the calls below need for this configuration
+ * (0 if the configuration is invalid; see moe_get_last_error).  The
+ * workspace holds logits, routing, the dispatch plan, the gathered
+ * activations and the intermediate expert outputs; it must be 256-byte
+ * aligned. */
+size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Router: steps a1-a4.  Page: mlqm.cn 稀疏激活 (sigmoid, noaux_tc,
+ * norm_topk_prob); Dots1 table (n_group, topk_group, routed_scaling_factor);
+ * Deep Dive §3.1 (gate, top-k, renormalise).
+ *   x        bf16 [T, H]        tokens
+ *   w_router bf16 [E, H]        gate weight (no bias term)
+ *   bias     fp32 [E]           noaux_tc selection bias
+ *   logits   fp32 [T, E]  out   x W_g^T (fp32 accumulation)
+ *   topk_idx int32 [T, k] out   chosen experts in slot order
+ *   topk_w   fp32 [T, k]  out   routing weights
+ *   ws       workspace (moe_workspace_size bytes)                          */
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_router,
+                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router selection alone (steps a2-a4) from given fp32 logits [T, E]: the
+ * same outputs as moe_route without the GEMM.  No workspace. */
+moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
+                                   const float* bias, int32_t* topk_idx, float* topk_w,
+                                   moe_stream_t stream);
+
+/* Dispatch order: step a5 (Deep Dive §8.2 "dispatch").  A counting sort of
+ * the T*k (token, slot) pairs by expert, stable in t*k + j, so that the rows
+ * of one expert are contiguous and in token order.
+ *   topk_idx int32 [T, k]       from moe_route
+ *   offsets  int32 [E + 1] out  first sorted row of each expert; offsets[E] = T*k
+ *   rows     int32 [T*k]   out  source token of each sorted row
+ *   pos      int32 [T*k]   out  sorted row of slot t*k + j                   */
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* offsets,
+                         int32_t* rows, int32_t* pos, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* Expert FFNs: steps a6-a8 (Deep Dive §8.2 "gmm1 -> swiglu -> gmm2"; Dots1
+ * packed gate_up_proj).  Gathers the sorted rows, runs every expert's
+ * SwiGLU on its rows as one grouped GEMM pair on the tensor cores, and
+ * scales each routed row by its routing weight.
+ *   x, offsets, rows, pos, topk_w   as above
+ *   w13   bf16 [E, 2I, H]   per expert: gate rows 0..I-1, up rows I..2I-1
+ *   w2    bf16 [E, H, I]    per expert down projection
+ *   w13s  bf16 [2 Is, H]    shared expert gate/up (Is = n_shared * I)
+ *   w2s   bf16 [H, Is]      shared expert down
+ *   y     bf16 [T*k, H] out w_j * SwiGLU_{idx_j}(x_t) at row pos[t*k + j]
+ *   y_shared bf16 [T, H] out  SwiGLU_shared(x) (may be NULL iff n_shared == 0)
+ * The *_scale arguments are reserved for block-scaled weights and must be
+ * NULL for MOE_DTYPE_BF16.                                                  */
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_t* offsets,
+                            const int32_t* rows, const int32_t* pos, const float* topk_w,
+                            const void* w13, const float* w13_scale, const void* w2,
+                            const float* w2_scale, const void* w13s, const float* w13s_scale,
+                            const void* w2s, const float* w2s_scale, void* y, void* y_shared,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine: step a9 (Deep Dive §3.3 "Weighted sum" then shared "add").
+ * out_t = sum_{j=0..k-1} y[pos[t*k + j]] + y_shared_t, summed in fp32 in
+ * that fixed order (no atomics: bitwise reproducible), rounded once to bf16.
+ *   y bf16 [T*k, H], pos int32 [T*k], y_shared bf16 [T, H] or NULL,
+ *   out bf16 [T, H]                                                        */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* pos,
+                         const void* y_shared, void* out, moe_stream_t stream);
+
+/* The whole layer (steps a1-a9) on one stream, intermediates in `ws`.
+ * Arguments as above; out bf16 [T, H].  stage_events: NULL, or
+ * MOE_NUM_STAGES + 1 cudaEvent_t handles recorded at the stage boundaries
+ * (for timing; the library only records them). */
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_router,
+                         const float* bias, const void* w13, const float* w13_scale,
+                         const void* w2, const float* w2_scale, const void* w13s,
+                         const float* w13s_scale, const void* w2s, const float* w2s_scale,
+                         void* out, void* ws, size_t ws_bytes, void* const* stage_events,
+                         moe_stream_t stream);
+
+/* Device byte offsets, inside the workspace, of the intermediates that
+ * moe_forward leaves there (for inspection and tests):
+ * which = 0 logits fp32 [T,E], 1 topk_idx int32 [T,k], 2 topk_w fp32 [T,k],
+ * 3 offsets int32 [E+1], 4 rows int32 [T*k], 5 pos int32 [T*k],
+ * 6 y bf16 [T*k,H], 7 y_shared bf16 [T,H].  Returns (size_t)-1 if invalid. */
+size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
+
+/* Synchronise `stream`, read and clear the device status word in `ws`.
+ * Returns MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait.  */
+moe_status_t moe_check_device_status(void* ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

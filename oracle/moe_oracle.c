@@ -31,6 +31,7 @@
  *  - group score = sum of the top `group_topn` (2) choice keys in a group of
  *    E/n_group contiguous experts; keep the top `topk_group` groups;
  *  - ties in every top-k: larger key first, equal keys -> lower index first;
+ *    a NaN key (NaN logit or bias) counts as -infinity;
  *  - weights: s_j / (s_0 + s_1 + ... + s_{k-1}) summed in slot order in fp32,
  *    then times routed_scaling_factor;
  *  - expert FFN is SwiGLU: down(SiLU(gate x) * up x), gate rows 0..I-1 and up
@@ -216,6 +217,7 @@ int orc_route(const orc_config* cfg, const float* logits, const float* bias, int
             for (int e = 0; e < E; ++e) {
                 s[e] = orc_sigmoid(logits[(size_t)t * E + e]);
                 c[e] = s[e] + bias[e]; /* the bias only steers the choice */
+                if (c[e] != c[e]) c[e] = -INFINITY; /* NaN ranks below numbers */
                 eligible[e] = 1;
                 taken[e] = 0;
             }
@@ -233,7 +235,7 @@ int orc_route(const orc_config* cfg, const float* logits, const float* bias, int
                     }
                     float acc = top[0];
                     for (int j = 1; j < tn; ++j) acc = acc + top[j];
-                    gscore[g] = acc;
+                    gscore[g] = acc != acc ? -INFINITY : acc;
                     for (int e = g * gsize; e < (g + 1) * gsize; ++e) used[e] = 0;
                 }
                 for (int g = 0; g < G; ++g) gkeep[g] = 0;

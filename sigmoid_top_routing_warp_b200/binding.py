@@ -1,0 +1,218 @@
+"""ctypes binding of libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers
+together with the current CUDA stream; every step of the layer runs in the
+library's kernels.  There is no fallback: if the shared library is missing,
+importing this module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError("libmoe_b200.so is not built (%s); build it with "
+                      "`python -m sigmoid_top_routing_warp_b200.build`" % _LIB_PATH)
+_lib = ctypes.CDLL(_LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
+    MOE_ERR_TIMEOUT = range(6)
+MOE_DTYPE_BF16 = 0
+MOE_NUM_STAGES = 6
+STAGE_NAMES = ("router_gemm", "router_select", "dispatch", "gate_up_swiglu", "down_weighted",
+               "combine")
+WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "pos": 5,
+            "y": 6, "y_shared": 7}
+
+# Every symbol include/moe.h declares.
+EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
+            "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
+            "moe_forward", "moe_check_device_status")
+
+
+class MoeConfigC(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("group_topn", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+@dataclass
+class MoeConfig:
+    """moe_config_t (field names follow the Dots1 / DeepSeek-V3 config)."""
+    T: int
+    H: int
+    E: int
+    k: int
+    I: int
+    n_shared: int = 1
+    n_group: int = 1
+    topk_group: int = 1
+    group_topn: int = 2
+    norm_topk_prob: bool = True
+    routed_scaling_factor: float = 1.0
+    dtype: int = MOE_DTYPE_BF16
+    flags: int = 0
+
+    def c(self) -> MoeConfigC:
+        return MoeConfigC(self.T, self.H, self.E, self.k, self.I, self.n_shared, self.n_group,
+                          self.topk_group, self.group_topn, int(bool(self.norm_topk_prob)),
+                          float(self.routed_scaling_factor), self.dtype, self.flags)
+
+    @property
+    def Is(self) -> int:
+        return self.n_shared * self.I
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed (status %d): %s" % (where, status, get_last_error()))
+
+
+_P = ctypes.c_void_p
+_CFG = ctypes.POINTER(MoeConfigC)
+_lib.moe_get_last_error.restype = ctypes.c_char_p
+_lib.moe_get_last_error.argtypes = []
+_lib.moe_workspace_size.restype = ctypes.c_size_t
+_lib.moe_workspace_size.argtypes = [_CFG]
+_lib.moe_workspace_offset.restype = ctypes.c_size_t
+_lib.moe_workspace_offset.argtypes = [_CFG, ctypes.c_int32]
+_lib.moe_route.restype = ctypes.c_int
+_lib.moe_route.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.moe_route_from_logits.restype = ctypes.c_int
+_lib.moe_route_from_logits.argtypes = [_CFG, _P, _P, _P, _P, _P]
+_lib.moe_permute.restype = ctypes.c_int
+_lib.moe_permute.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.moe_expert_ffn.restype = ctypes.c_int
+_lib.moe_expert_ffn.argtypes = [_CFG] + [_P] * 16 + [ctypes.c_size_t, _P]
+_lib.moe_combine.restype = ctypes.c_int
+_lib.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
+_lib.moe_forward.restype = ctypes.c_int
+_lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
+_lib.moe_check_device_status.restype = ctypes.c_int
+_lib.moe_check_device_status.argtypes = [_P, _P]
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def get_last_error() -> str:
+    return _lib.moe_get_last_error().decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != MOE_OK:
+        raise MoeError(st, where)
+
+
+def workspace_size(cfg: MoeConfig) -> int:
+    c = cfg.c()
+    n = _lib.moe_workspace_size(ctypes.byref(c))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    return n
+
+
+def workspace_offset(cfg: MoeConfig, item: str) -> int:
+    c = cfg.c()
+    off = _lib.moe_workspace_offset(ctypes.byref(c), WS_ITEMS[item])
+    if off == ctypes.c_size_t(-1).value:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_workspace_offset")
+    return off
+
+
+def alloc_workspace(cfg: MoeConfig, device="cuda") -> torch.Tensor:
+    """A zeroed workspace of moe_workspace_size bytes (256-byte aligned)."""
+    return torch.zeros(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg, x, w_router, bias, logits, topk_idx, topk_w, ws, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_route(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits),
+                          _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_route")
+
+
+def moe_route_from_logits(cfg, logits, bias, topk_idx, topk_w, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_route_from_logits(ctypes.byref(c), _ptr(logits), _ptr(bias), _ptr(topk_idx),
+                                      _ptr(topk_w), _stream(stream)), "moe_route_from_logits")
+
+
+def moe_permute(cfg, topk_idx, offsets, rows, pos, ws, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_permute(ctypes.byref(c), _ptr(topk_idx), _ptr(offsets), _ptr(rows), _ptr(pos),
+                            _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(cfg, x, offsets, rows, pos, topk_w, w13, w2, w13s, w2s, y, y_shared, ws,
+                   stream=None, w13_scale=None, w2_scale=None, w13s_scale=None, w2s_scale=None):
+    c = cfg.c()
+    _check(_lib.moe_expert_ffn(ctypes.byref(c), _ptr(x), _ptr(offsets), _ptr(rows), _ptr(pos),
+                               _ptr(topk_w), _ptr(w13), _ptr(w13_scale), _ptr(w2), _ptr(w2_scale),
+                               _ptr(w13s), _ptr(w13s_scale), _ptr(w2s), _ptr(w2s_scale), _ptr(y),
+                               _ptr(y_shared), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(cfg, y, pos, y_shared, out, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_combine(ctypes.byref(c), _ptr(y), _ptr(pos), _ptr(y_shared), _ptr(out),
+                            _stream(stream)), "moe_combine")
+
+
+def moe_forward(cfg, x, w_router, bias, w13, w2, w13s, w2s, out, ws, stream=None,
+                stage_events=None, w13_scale=None, w2_scale=None, w13s_scale=None,
+                w2s_scale=None):
+    """The whole layer.  stage_events: None or MOE_NUM_STAGES + 1 recorded
+    torch.cuda.Event objects (enable_timing=True) to time the stages."""
+    c = cfg.c()
+    ev = None
+    if stage_events is not None:
+        assert len(stage_events) == MOE_NUM_STAGES + 1
+        ev = (ctypes.c_void_p * (MOE_NUM_STAGES + 1))(*[e.cuda_event for e in stage_events])
+    _check(_lib.moe_forward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13),
+                            _ptr(w13_scale), _ptr(w2), _ptr(w2_scale), _ptr(w13s),
+                            _ptr(w13s_scale), _ptr(w2s), _ptr(w2s_scale), _ptr(out), _ptr(ws),
+                            ws.numel(), ev, _stream(stream)), "moe_forward")
+
+
+def moe_check_device_status(ws, stream=None):
+    _check(_lib.moe_check_device_status(_ptr(ws), _stream(stream)), "moe_check_device_status")
+
+
+def ws_view(ws: torch.Tensor, cfg: MoeConfig, item: str) -> torch.Tensor:
+    """A typed view of an intermediate moe_forward leaves in the workspace."""
+    off = workspace_offset(cfg, item)
+    T, E, k, H = cfg.T, cfg.E, cfg.k, cfg.H
+    shape, dt = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32),
+                 "topk_w": ((T, k), torch.float32), "offsets": ((E + 1,), torch.int32),
+                 "rows": ((T * k,), torch.int32), "pos": ((T * k,), torch.int32),
+                 "y": ((T * k, H), torch.bfloat16), "y_shared": ((T, H), torch.bfloat16)}[item]
+    n = 1
+    for d in shape:
+        n *= d
+    nbytes = n * torch.empty((), dtype=dt).element_size()
+    return ws[off:off + nbytes].view(dt).view(shape)

@@ -1,0 +1,561 @@
+// api.cu -- the C ABI declared in include/moe.h: argument checks, workspace
+// layout, TMA tensor maps and the launch sequence of the MoE FFN layer.
+// The library never allocates device memory; every buffer is the caller's.
+#include "moe.h"
+#include "kernels.cuh"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MOE_CUDA(call, what)                            \
+    do {                                                \
+        cudaError_t e_ = (call);                        \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ config
+moe_status_t check_config(const moe_config_t* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+    if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d must be >= 0", c->T);
+    if (c->dtype != MOE_DTYPE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "dtype %d not supported", c->dtype);
+    if (c->H <= 0 || c->H % 128)
+        return fail(MOE_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 128", c->H);
+    if (c->E < 32 || c->E > 1024 || c->E % 32)
+        return fail(MOE_ERR_UNSUPPORTED, "E=%d must be a multiple of 32 in [32, 1024]", c->E);
+    switch (c->E / 32) {
+        case 1: case 2: case 3: case 4: case 5: case 6: case 8: case 10: case 12: case 16:
+        case 24: case 32: break;
+        default: return fail(MOE_ERR_UNSUPPORTED, "E=%d: E/32 must be one of 1-6,8,10,12,16,24,32", c->E);
+    }
+    if (c->k < 1 || c->k > 32 || c->k > c->E)
+        return fail(MOE_ERR_INVALID_ARG, "k=%d must be in [1, min(E, 32)]", c->k);
+    if (c->I <= 0 || c->I % 128)
+        return fail(MOE_ERR_UNSUPPORTED, "I=%d must be a positive multiple of 128", c->I);
+    if (c->n_shared < 0 || (long long)c->n_shared * c->I > (1 << 20))
+        return fail(MOE_ERR_INVALID_ARG, "n_shared=%d out of range", c->n_shared);
+    const int G = c->n_group, tg = c->topk_group;
+    if (G < 1 || G > 32 || c->E % G)
+        return fail(MOE_ERR_INVALID_ARG, "n_group=%d must divide E and be in [1, 32]", G);
+    if (tg < 1 || tg > G)
+        return fail(MOE_ERR_INVALID_ARG, "topk_group=%d must be in [1, n_group]", tg);
+    if (G > 1 && (c->group_topn < 1 || c->group_topn > c->E / G))
+        return fail(MOE_ERR_INVALID_ARG, "group_topn=%d must be in [1, E/n_group]", c->group_topn);
+    if (c->k > tg * (c->E / G))
+        return fail(MOE_ERR_INVALID_ARG, "k=%d exceeds the experts of topk_group groups", c->k);
+    if ((long long)c->T * c->k > (1ll << 30) / 8)
+        return fail(MOE_ERR_UNSUPPORTED, "T*k=%lld too large", (long long)c->T * c->k);
+    return MOE_OK;
+}
+
+// Token-tile width of the expert GEMMs: the MMA N operand.  Decode-sized
+// batches (a few tokens per expert) use 16; prefill-sized batches use 128.
+int expert_bn(const moe_config_t* c) {
+    const double avg = c->E ? (double)c->T * c->k / c->E : 0.0;
+    return avg <= 24.0 ? 16 : avg <= 96.0 ? 64 : 128;
+}
+int router_bn(const moe_config_t* c) { return c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128; }
+
+struct Layout {
+    size_t status, logits, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash, y,
+        ysh, total;
+};
+
+Layout layout(const moe_config_t* c) {
+    Layout L{};
+    const size_t T = c->T, E = c->E, k = c->k, H = c->H, I = c->I, Is = (size_t)c->n_shared * c->I;
+    const size_t n = T * k;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    };
+    L.status = take(256);
+    L.logits = take(T * E * 4);
+    L.idx = take(n * 4);
+    L.w = take(n * 4);
+    L.offsets = take((E + 1) * 4);
+    L.rows = take(n * 4);
+    L.pos = take(n * 4);
+    L.wperm = take(n * 4);
+    L.tokstart = take((E + 1) * 4);
+    L.chunk = take((size_t)moe::permute_chunks((int)n) * E * 4);
+    L.xperm = take(n * H * 2);
+    L.a = take(n * I * 2);
+    L.ash = take(T * Is * 2);
+    L.y = take(n * H * 2);
+    L.ysh = take(T * H * 2);
+    L.total = off;
+    return L;
+}
+
+template <typename Tp>
+Tp* at(void* ws, size_t off) {
+    return reinterpret_cast<Tp*>(static_cast<char*>(ws) + off);
+}
+
+moe_status_t check_ws(const moe_config_t* c, void* ws, size_t ws_bytes) {
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u)
+        return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t need = layout(c).total;
+    if (ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 row-major [rows, cols] as a 2-D tensor, box {64 columns, box_rows},
+// 128-byte swizzle (the K-major layout the tensor-core descriptors expect).
+moe_status_t make_map(CUtensorMap* m, const void* ptr, size_t rows, size_t cols, int box_rows,
+                      const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
+
+moe_status_t sm_count(int* n) {
+    int dev = 0;
+    MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    MOE_CUDA(cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev), "SM count");
+    return MOE_OK;
+}
+
+#define MOE_TRY(x)                          \
+    do {                                    \
+        moe_status_t st_ = (x);             \
+        if (st_ != MOE_OK) return st_;      \
+    } while (0)
+
+// ------------------------------------------------------------------ stages
+moe_status_t run_router_gemm(const moe_config_t* c, const void* x, const void* wg, float* logits,
+                             int* status, cudaStream_t s) {
+    moe::GemmParams P;
+    memset(&P, 0, sizeof(P));
+    const int bn = router_bn(c);
+    moe::GemmProblem& p = P.p[0];
+    MOE_TRY(make_map(&p.tw, wg, c->E, c->H, 128, "w_router"));
+    MOE_TRY(make_map(&p.tx, x, c->T, c->H, bn, "x"));
+    p.seg = nullptr;
+    p.tok_start = nullptr;
+    p.n_exp = 1;
+    p.n_rows = c->T;
+    p.K = c->H;
+    p.n_feat = c->E;
+    p.w_rows = c->E;
+    p.out = logits;
+    p.ld_out = c->E;
+    p.row_w = nullptr;
+    P.n_problems = 1;
+    P.status = status;
+    int sms = 0;
+    MOE_TRY(sm_count(&sms));
+    const int tiles = ((c->E + 127) / 128) * ((c->T + bn - 1) / bn);
+    const int grid = tiles < sms ? tiles : sms;
+    MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_F32, bn, P, grid, s), "router GEMM launch");
+    return MOE_OK;
+}
+
+moe_status_t run_select(const moe_config_t* c, const float* logits, const float* bias,
+                        int32_t* idx, float* w, cudaStream_t s) {
+    moe::RouteArgs a;
+    a.logits = logits;
+    a.bias = bias;
+    a.idx = idx;
+    a.w = w;
+    a.T = c->T;
+    a.E = c->E;
+    a.k = c->k;
+    a.n_group = c->n_group;
+    a.topk_group = c->topk_group;
+    a.group_topn = c->group_topn;
+    a.norm = c->norm_topk_prob != 0;
+    a.rsf = c->routed_scaling_factor;
+    MOE_CUDA(moe::launch_route_select(a, s), "router selection launch");
+    return MOE_OK;
+}
+
+moe_status_t run_permute(const moe_config_t* c, const int32_t* idx, int32_t* offsets,
+                         int32_t* rows, int32_t* pos, void* ws, cudaStream_t s) {
+    moe::PermuteArgs a;
+    a.idx = idx;
+    a.offsets = offsets;
+    a.rows = rows;
+    a.pos = pos;
+    a.chunk_base = at<int32_t>(ws, layout(c).chunk);
+    a.T = c->T;
+    a.k = c->k;
+    a.E = c->E;
+    MOE_CUDA(moe::launch_permute(a, s), "permute launch");
+    return MOE_OK;
+}
+
+struct Weights {
+    const void *w13, *w2, *w13s, *w2s;
+};
+
+moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t* offsets,
+                            const int32_t* pos, const float* topk_w, const Weights& W, void* y,
+                            void* y_shared, void* ws, cudaStream_t s, cudaEvent_t ev_mid,
+                            cudaEvent_t ev_gemm2) {
+    const Layout L = layout(c);
+    const int bn = expert_bn(c);
+    const int n = c->T * c->k;
+    const int Is = c->n_shared * c->I;
+
+    moe::GatherArgs g;
+    g.x = static_cast<const uint16_t*>(x);
+    g.pos = pos;
+    g.topk_w = topk_w;
+    g.offsets = offsets;
+    g.x_perm = at<uint16_t>(ws, L.xperm);
+    g.w_perm = at<float>(ws, L.wperm);
+    g.tok_start = at<int32_t>(ws, L.tokstart);
+    g.T = c->T;
+    g.k = c->k;
+    g.H = c->H;
+    g.E = c->E;
+    g.bn = bn;
+    MOE_CUDA(moe::launch_gather(g, s), "gather launch");
+    if (ev_mid) MOE_CUDA(cudaEventRecord(ev_mid, s), "event record");
+
+    int sms = 0;
+    MOE_TRY(sm_count(&sms));
+    int* status = at<int>(ws, L.status);
+
+    // gate/up GEMM + SwiGLU: routed experts, then the shared expert
+    moe::GemmParams P1;
+    memset(&P1, 0, sizeof(P1));
+    {
+        moe::GemmProblem& p = P1.p[0];
+        MOE_TRY(make_map(&p.tw, W.w13, (size_t)c->E * 2 * c->I, c->H, 128, "w13"));
+        MOE_TRY(make_map(&p.tx, g.x_perm, n, c->H, bn, "gathered x"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->H;
+        p.n_feat = c->I;
+        p.w_rows = 2 * c->I;
+        p.out = at<void>(ws, L.a);
+        p.ld_out = c->I;
+        P1.n_problems = 1;
+        if (Is > 0) {
+            moe::GemmProblem& q = P1.p[1];
+            MOE_TRY(make_map(&q.tw, W.w13s, (size_t)2 * Is, c->H, 128, "w13s"));
+            MOE_TRY(make_map(&q.tx, x, c->T, c->H, bn, "x"));
+            q.seg = nullptr;
+            q.tok_start = nullptr;
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = c->H;
+            q.n_feat = Is;
+            q.w_rows = 2 * Is;
+            q.out = at<void>(ws, L.ash);
+            q.ld_out = Is;
+            P1.n_problems = 2;
+        }
+        P1.status = status;
+    }
+    MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_SWIGLU, bn, P1, sms, s), "gate/up GEMM launch");
+    if (ev_gemm2) MOE_CUDA(cudaEventRecord(ev_gemm2, s), "event record");
+
+    // down GEMM x routing weight: routed experts, then the shared expert
+    moe::GemmParams P2;
+    memset(&P2, 0, sizeof(P2));
+    {
+        moe::GemmProblem& p = P2.p[0];
+        MOE_TRY(make_map(&p.tw, W.w2, (size_t)c->E * c->H, c->I, 128, "w2"));
+        MOE_TRY(make_map(&p.tx, at<void>(ws, L.a), n, c->I, bn, "expert activations"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->I;
+        p.n_feat = c->H;
+        p.w_rows = c->H;
+        p.out = y;
+        p.ld_out = c->H;
+        p.row_w = g.w_perm;
+        P2.n_problems = 1;
+        if (Is > 0) {
+            moe::GemmProblem& q = P2.p[1];
+            MOE_TRY(make_map(&q.tw, W.w2s, c->H, Is, 128, "w2s"));
+            MOE_TRY(make_map(&q.tx, at<void>(ws, L.ash), c->T, Is, bn, "shared activations"));
+            q.seg = nullptr;
+            q.tok_start = nullptr;
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = Is;
+            q.n_feat = c->H;
+            q.w_rows = c->H;
+            q.out = y_shared;
+            q.ld_out = c->H;
+            q.row_w = nullptr;
+            P2.n_problems = 2;
+        }
+        P2.status = status;
+    }
+    MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_SCALE, bn, P2, sms, s), "down GEMM launch");
+    return MOE_OK;
+}
+
+moe_status_t run_combine(const moe_config_t* c, const void* y, const int32_t* pos,
+                         const void* y_shared, void* out, cudaStream_t s) {
+    moe::CombineArgs a;
+    a.y = static_cast<const uint16_t*>(y);
+    a.pos = pos;
+    a.y_shared = static_cast<const uint16_t*>(y_shared);
+    a.out = static_cast<uint16_t*>(out);
+    a.T = c->T;
+    a.k = c->k;
+    a.H = c->H;
+    MOE_CUDA(moe::launch_combine(a, s), "combine launch");
+    return MOE_OK;
+}
+
+moe_status_t need(const void* p, const char* name) {
+    return p ? MOE_OK : fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+}
+
+moe_status_t need16(const void* p, const char* name) {
+    MOE_TRY(need(p, name));
+    return aligned16(p) ? MOE_OK : fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+}
+
+moe_status_t check_scales(const float* a, const float* b, const float* c2, const float* d) {
+    if (a || b || c2 || d)
+        return fail(MOE_ERR_INVALID_ARG, "weight scales must be NULL for bf16 weights");
+    return MOE_OK;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+extern "C" {
+
+const char* moe_get_last_error(void) { return g_err; }
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    return layout(cfg).total;
+}
+
+size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which) {
+    if (check_config(cfg) != MOE_OK) return (size_t)-1;
+    const Layout L = layout(cfg);
+    switch (which) {
+        case 0: return L.logits;
+        case 1: return L.idx;
+        case 2: return L.w;
+        case 3: return L.offsets;
+        case 4: return L.rows;
+        case 5: return L.pos;
+        case 6: return L.y;
+        case 7: return L.ysh;
+        default: fail(MOE_ERR_INVALID_ARG, "unknown workspace item %d", which); return (size_t)-1;
+    }
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_router,
+                       const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need16(w_router, "w_router"));
+    MOE_TRY(need(bias, "bias"));
+    MOE_TRY(need(logits, "logits"));
+    MOE_TRY(need(topk_idx, "topk_idx"));
+    MOE_TRY(need(topk_w, "topk_w"));
+    if (cfg->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MOE_TRY(run_router_gemm(cfg, x, w_router, logits, at<int>(ws, layout(cfg).status), s));
+    return run_select(cfg, logits, bias, topk_idx, topk_w, s);
+}
+
+moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
+                                   const float* bias, int32_t* topk_idx, float* topk_w,
+                                   moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(need(logits, "logits"));
+    MOE_TRY(need(bias, "bias"));
+    MOE_TRY(need(topk_idx, "topk_idx"));
+    MOE_TRY(need(topk_w, "topk_w"));
+    if (cfg->T == 0) return MOE_OK;
+    return run_select(cfg, logits, bias, topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* offsets,
+                         int32_t* rows, int32_t* pos, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    MOE_TRY(need(topk_idx, "topk_idx"));
+    MOE_TRY(need(offsets, "offsets"));
+    MOE_TRY(need(rows, "rows"));
+    MOE_TRY(need(pos, "pos"));
+    return run_permute(cfg, topk_idx, offsets, rows, pos, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_t* offsets,
+                            const int32_t* rows, const int32_t* pos, const float* topk_w,
+                            const void* w13, const float* w13_scale, const void* w2,
+                            const float* w2_scale, const void* w13s, const float* w13s_scale,
+                            const void* w2s, const float* w2s_scale, void* y, void* y_shared,
+                            void* ws, size_t ws_bytes, moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    MOE_TRY(check_scales(w13_scale, w2_scale, w13s_scale, w2s_scale));
+    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need(offsets, "offsets"));
+    MOE_TRY(need(rows, "rows"));
+    MOE_TRY(need(pos, "pos"));
+    MOE_TRY(need(topk_w, "topk_w"));
+    MOE_TRY(need16(w13, "w13"));
+    MOE_TRY(need16(w2, "w2"));
+    MOE_TRY(need16(y, "y"));
+    if (cfg->n_shared > 0) {
+        MOE_TRY(need16(w13s, "w13s"));
+        MOE_TRY(need16(w2s, "w2s"));
+        MOE_TRY(need16(y_shared, "y_shared"));
+    }
+    if (cfg->T == 0) return MOE_OK;
+    Weights W{w13, w2, w13s, w2s};
+    return run_expert_ffn(cfg, x, offsets, pos, topk_w, W, y, y_shared, ws,
+                          static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* pos,
+                         const void* y_shared, void* out, moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(need16(y, "y"));
+    MOE_TRY(need(pos, "pos"));
+    MOE_TRY(need16(out, "out"));
+    if (y_shared && !aligned16(y_shared))
+        return fail(MOE_ERR_INVALID_ARG, "y_shared must be 16-byte aligned");
+    if (cfg->T == 0) return MOE_OK;
+    return run_combine(cfg, y, pos, y_shared, out, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_router,
+                         const float* bias, const void* w13, const float* w13_scale,
+                         const void* w2, const float* w2_scale, const void* w13s,
+                         const float* w13s_scale, const void* w2s, const float* w2s_scale,
+                         void* out, void* ws, size_t ws_bytes, void* const* stage_events,
+                         moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    MOE_TRY(check_scales(w13_scale, w2_scale, w13s_scale, w2s_scale));
+    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need16(w_router, "w_router"));
+    MOE_TRY(need(bias, "bias"));
+    MOE_TRY(need16(w13, "w13"));
+    MOE_TRY(need16(w2, "w2"));
+    MOE_TRY(need16(out, "out"));
+    if (cfg->n_shared > 0) {
+        MOE_TRY(need16(w13s, "w13s"));
+        MOE_TRY(need16(w2s, "w2s"));
+    }
+    if (cfg->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
+    if (stage_events)
+        for (int i = 0; i <= MOE_NUM_STAGES; ++i) ev[i] = static_cast<cudaEvent_t>(stage_events[i]);
+    auto mark = [&](int i) -> moe_status_t {
+        if (ev[i]) MOE_CUDA(cudaEventRecord(ev[i], s), "event record");
+        return MOE_OK;
+    };
+    const Layout L = layout(cfg);
+    float* logits = at<float>(ws, L.logits);
+    int32_t* idx = at<int32_t>(ws, L.idx);
+    float* w = at<float>(ws, L.w);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* pos = at<int32_t>(ws, L.pos);
+    void* y = at<void>(ws, L.y);
+    void* ysh = cfg->n_shared > 0 ? at<void>(ws, L.ysh) : nullptr;
+
+    MOE_TRY(mark(0));
+    MOE_TRY(run_router_gemm(cfg, x, w_router, logits, at<int>(ws, L.status), s));
+    MOE_TRY(mark(1));
+    MOE_TRY(run_select(cfg, logits, bias, idx, w, s));
+    MOE_TRY(mark(2));
+    MOE_TRY(run_permute(cfg, idx, offsets, at<int32_t>(ws, L.rows), pos, ws, s));
+    Weights W{w13, w2, w13s, w2s};
+    MOE_TRY(run_expert_ffn(cfg, x, offsets, pos, w, W, y, ysh, ws, s, ev[3], ev[4]));
+    MOE_TRY(mark(5));
+    MOE_TRY(run_combine(cfg, y, pos, ysh, out, s));
+    return mark(6);
+}
+
+moe_status_t moe_check_device_status(void* ws, moe_stream_t stream) {
+    g_err[0] = 0;
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    int word = 0;
+    MOE_CUDA(cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost), "status read");
+    const int zero = 0;
+    MOE_CUDA(cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice), "status clear");
+    if (word & moe::DEV_STATUS_TIMEOUT)
+        return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", word);
+    return MOE_OK;
+}
+
+}  // extern "C"

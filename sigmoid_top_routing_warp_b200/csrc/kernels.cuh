@@ -1,0 +1,89 @@
+// kernels.cuh -- launch interface between the C-ABI layer (api.cu) and the
+// CUDA kernels of the MoE FFN layer.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device status word bits (stored in the workspace).
+enum : int { DEV_STATUS_TIMEOUT = 1 };
+
+// ---------------------------------------------------------------- router
+struct RouteArgs {
+    const float* logits;  // [T, E]
+    const float* bias;    // [E]
+    int32_t* idx;         // [T, k]
+    float* w;             // [T, k]
+    int T, E, k, n_group, topk_group, group_topn, norm;
+    float rsf;
+};
+cudaError_t launch_route_select(const RouteArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- dispatch
+struct PermuteArgs {
+    const int32_t* idx;   // [T, k]
+    int32_t* offsets;     // [E + 1]
+    int32_t* rows;        // [T*k]
+    int32_t* pos;         // [T*k]
+    int32_t* chunk_base;  // [n_chunks, E] scratch (large path)
+    int T, k, E;
+};
+int permute_chunks(int n_slots);  // chunks of the multi-block path (0: single block)
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+
+struct GatherArgs {
+    const uint16_t* x;        // bf16 [T, H]
+    const int32_t* pos;       // [T*k]
+    const float* topk_w;      // [T*k]
+    const int32_t* offsets;   // [E + 1]
+    uint16_t* x_perm;         // bf16 [T*k, H]
+    float* w_perm;            // [T*k]
+    int32_t* tok_start;       // [E + 1] token-tile prefix, tiles of bn rows
+    int T, k, H, E, bn;
+};
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+    const uint16_t* y;        // bf16 [T*k, H]
+    const int32_t* pos;       // [T*k]
+    const uint16_t* y_shared; // bf16 [T, H] or null
+    uint16_t* out;            // bf16 [T, H]
+    int T, k, H;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- grouped GEMM
+enum Epilogue : int { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_SCALE = 2 };
+
+// One problem of a grouped GEMM launch, in "weights x tokens" orientation:
+// for every expert e and every 128-row tile of its weight matrix,
+//   D[f, r] = sum_k W_e[f, k] * X[r, k]  over the token rows r of expert e,
+// written transposed to out[r, f].
+struct GemmProblem {
+    CUtensorMap tw;           // weights, bf16 2-D [rows, K], box {64, 128}
+    CUtensorMap tx;           // activations, bf16 2-D [rows, K], box {64, bn}
+    const int32_t* seg;       // [n_exp + 1] token-row offsets, or null: rows [0, n_rows)
+    const int32_t* tok_start; // [n_exp + 1] token-tile prefix, or null with seg
+    int n_exp;
+    int n_rows;               // used when seg is null
+    int K;                    // multiple of 64
+    int n_feat;               // output features per expert
+    int w_rows;               // weight rows per expert
+    void* out;                // [rows, ld_out] (fp32 for EPI_F32, bf16 otherwise)
+    int ld_out;
+    const float* row_w;       // EPI_SCALE: per-row factor, or null (1.0)
+};
+
+struct GemmParams {
+    GemmProblem p[2];
+    int n_problems;
+    int* status;
+};
+
+// bn: token tile (16, 64 or 128).  grid: persistent CTAs.
+cudaError_t launch_grouped_gemm(int epi, int bn, const GemmParams& params, int grid,
+                                cudaStream_t s);
+
+}  // namespace moe

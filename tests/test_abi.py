@@ -1,0 +1,96 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything.
+No GPU is needed (no call here reaches a CUDA launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sigmoid_top_routing_warp_b200 import build
+    build.build()
+    from sigmoid_top_routing_warp_b200 import binding
+    return binding
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(B):
+    names = header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(B.lib(), n), n
+    assert sorted(B.EXPORTED) == names
+
+
+def cfg(B, **kw):
+    base = dict(T=64, H=5120, E=256, k=8, I=1536, n_shared=1)
+    base.update(kw)
+    return B.MoeConfig(**base)
+
+
+def test_workspace_size_and_offsets(B):
+    c = cfg(B)
+    n = B.workspace_size(c)
+    T, E, k, H, I = 64, 256, 8, 5120, 1536
+    # at least the gathered activations, intermediates and outputs
+    assert n >= T * k * H * 2 * 2 + T * k * I * 2 + T * H * 2
+    offs = [B.workspace_offset(c, it) for it in B.WS_ITEMS]
+    assert all(o % 256 == 0 and o < n for o in offs)
+    assert len(set(offs)) == len(offs)
+    big = cfg(B, T=8192)
+    assert B.workspace_size(big) > n
+
+
+@pytest.mark.parametrize("kw", [dict(H=100), dict(E=33), dict(E=0), dict(k=0), dict(k=300),
+                                dict(I=100), dict(n_group=3), dict(n_group=8, topk_group=9),
+                                dict(n_group=8, topk_group=1, k=33), dict(T=-1), dict(dtype=7),
+                                dict(n_shared=-1)])
+def test_invalid_configs_rejected(B, kw):
+    with pytest.raises(B.MoeError):
+        B.workspace_size(cfg(B, **kw))
+    assert B.get_last_error() != ""
+
+
+def test_calls_reject_bad_arguments_before_launch(B):
+    c = cfg(B)
+    cc = c.c()
+    ws_bytes = B.workspace_size(c)
+    fake_ws = 1 << 20  # aligned, never dereferenced: validation fails first
+    L = B.lib()
+    st = L.moe_route(ctypes.byref(cc), None, None, None, None, None, None, fake_ws, ws_bytes,
+                     None)
+    assert st == B.MOE_ERR_INVALID_ARG and "x" in B.get_last_error()
+    st = L.moe_route(ctypes.byref(cc), 16, 16, 16, 16, 16, 16, fake_ws, ws_bytes - 1, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    st = L.moe_route(ctypes.byref(cc), 16, 16, 16, 16, 16, 16, fake_ws + 8, ws_bytes, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "aligned" in B.get_last_error()
+    st = L.moe_permute(ctypes.byref(cc), None, 16, 16, 16, fake_ws, ws_bytes, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    st = L.moe_combine(ctypes.byref(cc), 24, 16, None, 32, None)   # y misaligned
+    assert st == B.MOE_ERR_INVALID_ARG and "aligned" in B.get_last_error()
+    st = L.moe_forward(ctypes.byref(cc), *([16] * 4), 16, *([16] * 7), fake_ws, ws_bytes, None,
+                       None)  # a weight scale given for bf16 weights
+    assert st == B.MOE_ERR_INVALID_ARG and "scale" in B.get_last_error()
+    st = L.moe_forward(None, *([16] * 12), fake_ws, ws_bytes, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    st = L.moe_check_device_status(None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(B):
+    c = cfg(B, T=0)
+    cc = c.c()
+    ws_bytes = B.workspace_size(c)
+    st = B.lib().moe_forward(ctypes.byref(cc), 16, 16, 16, 16, None, 16, None, 16, None, 16,
+                             None, 16, 1 << 20, ws_bytes, None, None)
+    assert st == B.MOE_OK
