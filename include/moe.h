@@ -145,6 +145,28 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32
                          int32_t* rows, int32_t* pos, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* Dispatch order like moe_permute, for callers that cannot allocate device
+ * memory at all (for example a plugin that its host framework hands only
+ * input and output buffers, or a runtime whose memory planner owns the whole
+ * HBM budget): no workspace argument.  The pages have no counterpart; this is
+ * a convenience of this library.  Its scratch is a fixed array of
+ * MOE_PERMUTE_NOALLOC_SCRATCH_INTS int32 values (256 KiB) in the library's
+ * device image, held by every GPU that loads the library until exit.
+ *   - Sizes whose multi-block pass needs more scratch than that
+ *     (ceil(T*k / 2048) * E entries when T*k > 4096) are rejected with
+ *     MOE_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (a one-time set-up per device); make that first
+ *     call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU race on
+ *     it and must not be issued.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ * Arguments and outputs as for moe_permute.                                 */
+#define MOE_PERMUTE_NOALLOC_SCRATCH_INTS 65536
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_idx,
+                                 int32_t* offsets, int32_t* rows, int32_t* pos,
+                                 moe_stream_t stream);
+
 /* Expert FFNs: steps a6-a8 (Deep Dive §8.2 "gmm1 -> swiglu -> gmm2"; Dots1
  * packed gate_up_proj).  Gathers the sorted rows, runs every expert's
  * SwiGLU on its rows as one grouped GEMM pair on the tensor cores, and

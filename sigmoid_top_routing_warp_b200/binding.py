@@ -31,7 +31,7 @@ WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "p
 # Every symbol include/moe.h declares.
 EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
-            "moe_forward", "moe_check_device_status")
+            "moe_forward", "moe_check_device_status", "moe_permute_noalloc")
 
 
 class MoeConfigC(ctypes.Structure):
@@ -96,6 +96,8 @@ _lib.moe_combine.restype = ctypes.c_int
 _lib.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_forward.restype = ctypes.c_int
 _lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
+_lib.moe_permute_noalloc.restype = ctypes.c_int
+_lib.moe_permute_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -165,6 +167,14 @@ def moe_permute(cfg, topk_idx, offsets, rows, pos, ws, stream=None):
     c = cfg.c()
     _check(_lib.moe_permute(ctypes.byref(c), _ptr(topk_idx), _ptr(offsets), _ptr(rows), _ptr(pos),
                             _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, topk_idx, offsets, rows, pos, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate
+    device memory; its scratch is a fixed array inside the library."""
+    c = cfg.c()
+    _check(_lib.moe_permute_noalloc(ctypes.byref(c), _ptr(topk_idx), _ptr(offsets), _ptr(rows),
+                                    _ptr(pos), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_expert_ffn(cfg, x, offsets, rows, pos, topk_w, w13, w2, w13s, w2s, y, y_shared, ws,

@@ -559,3 +559,11 @@ moe_status_t moe_check_device_status(void* ws, moe_stream_t stream) {
 }
 
 }  // extern "C"
+
+// Argument checks and the last-error message, shared with entry points that
+// live in other translation units of the library.
+namespace moe {
+moe_status_t api_check_config(const moe_config_t* c) { return check_config(c); }
+moe_status_t api_fail(moe_status_t st, const char* msg) { return fail(st, "%s", msg); }
+void api_clear_error() { g_err[0] = 0; }
+}  // namespace moe
