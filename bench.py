@@ -45,6 +45,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU work of the oracle sample")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's tokens")
+    ap.add_argument("--E", type=int, default=None,
+                    help="override the routed expert count (small profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -156,6 +160,17 @@ def layer_work(wl, touched: int):
 
 # ---------------------------------------------------------------- our arm
 
+def workload_of(args):
+    from dataclasses import replace
+    from sigmoid_top_routing_warp_b200 import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    if args.T is not None:
+        wl = replace(wl, T=args.T)
+    if args.E is not None:
+        wl = replace(wl, E=args.E, bias="uniform")
+    return wl
+
+
 def cfg_of(B, wl):
     return B.MoeConfig(T=wl.T, H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
                        n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
@@ -174,7 +189,7 @@ def run_ours(args, world, rank, local):
     from sigmoid_top_routing_warp_b200 import binding as B
     from sigmoid_top_routing_warp_b200 import workloads as W
 
-    wl = W.WORKLOADS[args.workload]
+    wl = workload_of(args)
     dev = torch.device("cuda", local if world > 1 else 0)
     inp = W.make_inputs(wl, device=dev, seed=wl.seed + rank)
     cfg = cfg_of(B, wl)
@@ -219,6 +234,10 @@ def run_ours(args, world, rank, local):
                        for i in range(K)])
     stage_ms = stages.mean(0)
 
+    if args.no_e2e:
+        return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
+                "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": None,
+                "launches": launches_per_step(B, cfg) * K, "B": B}
     # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
     x_host = inp["x"].cpu().pin_memory()
     out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
@@ -370,8 +389,9 @@ def main():
             "roofline": roof, "layer_roofline": layer,
             "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
             "gpu_launches": r["launches"], "clocks": r["clocks"],
-            "e2e": {"value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
+            "e2e": None if r["e2e_ms"] is None else {
+                "value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, sample = oracle_sample(wl, r["inp"], args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",

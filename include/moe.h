@@ -177,7 +177,9 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_id
  *   w13s  bf16 [2 Is, H]    shared expert gate/up (Is = n_shared * I)
  *   w2s   bf16 [H, Is]      shared expert down
  *   y     bf16 [T*k, H] out w_j * SwiGLU_{idx_j}(x_t) at row pos[t*k + j]
- *   y_shared bf16 [T, H] out  SwiGLU_shared(x) (may be NULL iff n_shared == 0)
+ *   y_shared fp32 [T, H] out  SwiGLU_shared(x) (may be NULL iff n_shared == 0);
+ *            kept in fp32 because, with weight 1, it is the largest term of
+ *            the combine and its rounding would dominate the output error
  * The *_scale arguments are reserved for block-scaled weights and must be
  * NULL for MOE_DTYPE_BF16.                                                  */
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_t* offsets,
@@ -190,7 +192,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_
 /* Combine: step a9 (Deep Dive §3.3 "Weighted sum" then shared "add").
  * out_t = sum_{j=0..k-1} y[pos[t*k + j]] + y_shared_t, summed in fp32 in
  * that fixed order (no atomics: bitwise reproducible), rounded once to bf16.
- *   y bf16 [T*k, H], pos int32 [T*k], y_shared bf16 [T, H] or NULL,
+ *   y bf16 [T*k, H], pos int32 [T*k], y_shared fp32 [T, H] or NULL,
  *   out bf16 [T, H]                                                        */
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* pos,
                          const void* y_shared, void* out, moe_stream_t stream);
@@ -210,7 +212,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
  * moe_forward leaves there (for inspection and tests):
  * which = 0 logits fp32 [T,E], 1 topk_idx int32 [T,k], 2 topk_w fp32 [T,k],
  * 3 offsets int32 [E+1], 4 rows int32 [T*k], 5 pos int32 [T*k],
- * 6 y bf16 [T*k,H], 7 y_shared bf16 [T,H].  Returns (size_t)-1 if invalid. */
+ * 6 y bf16 [T*k,H], 7 y_shared fp32 [T,H].  Returns (size_t)-1 if invalid. */
 size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
 
 /* Synchronise `stream`, read and clear the device status word in `ws`.

@@ -73,10 +73,11 @@ moe_status_t check_config(const moe_config_t* c) {
 }
 
 // Token-tile width of the expert GEMMs: the MMA N operand.  Decode-sized
-// batches (a few tokens per expert) use 16; prefill-sized batches use 128.
+// batches (a few tokens per expert) use 16 on single CTAs; prefill-sized
+// batches use 256-token tiles on CTA pairs.
 int expert_bn(const moe_config_t* c) {
     const double avg = c->E ? (double)c->T * c->k / c->E : 0.0;
-    return avg <= 24.0 ? 16 : avg <= 96.0 ? 64 : 128;
+    return avg <= 24.0 ? 16 : avg <= 96.0 ? 64 : moe::kPairTokens;
 }
 int router_bn(const moe_config_t* c) { return c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128; }
 
@@ -109,7 +110,7 @@ Layout layout(const moe_config_t* c) {
     L.a = take(n * I * 2);
     L.ash = take(T * Is * 2);
     L.y = take(n * H * 2);
-    L.ysh = take(T * H * 2);
+    L.ysh = take(T * H * 4);
     L.total = off;
     return L;
 }
@@ -160,6 +161,25 @@ moe_status_t make_map(CUtensorMap* m, const void* ptr, size_t rows, size_t cols,
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
+
+// Packed gate/up matrix [n_exp][2 n_feat][K] (bf16) as the 5-D view
+// {K, 8, 2, n_feat/8, n_exp}: a box {64, 8, 2, 8, 1} brings 64 features as
+// alternating 8-row gate and up blocks (128 rows of 128 bytes, 128-byte swizzle).
+moe_status_t make_map_gate_up_interleaved(CUtensorMap* m, const void* ptr, size_t n_exp,
+                                          size_t n_feat, size_t K, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[5] = {K, 8, 2, n_feat / 8, n_exp};
+    cuuint64_t strides[4] = {K * 2, n_feat * K * 2, 8 * K * 2, 2 * n_feat * K * 2};
+    cuuint32_t box[5] = {64, 8, 2, 8, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
@@ -246,6 +266,80 @@ struct Weights {
     const void *w13, *w2, *w13s, *w2s;
 };
 
+// Prefill-sized batches: both expert GEMMs on CTA pairs (256 x 256 tiles).
+moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const int32_t* offsets,
+                                  const Weights& W, void* y, void* y_shared, void* ws,
+                                  cudaStream_t s, cudaEvent_t ev_gemm2, const moe::GatherArgs& g,
+                                  int sms, int* status) {
+    const Layout L = layout(c);
+    const int n = c->T * c->k;
+    const int Is = c->n_shared * c->I;
+    const int half = moe::kPairTokens / 2;
+    moe::PairParams P1;
+    memset(&P1, 0, sizeof(P1));
+    {
+        moe::PairProblem& p = P1.p[0];
+        MOE_TRY(make_map_gate_up_interleaved(&p.tw, W.w13, c->E, c->I, c->H, "w13"));
+        MOE_TRY(make_map(&p.tx, g.x_perm, n, c->H, half, "gathered x"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->H;
+        p.n_feat = c->I;
+        p.out = at<void>(ws, L.a);
+        p.ld_out = c->I;
+        P1.n_problems = 1;
+        if (Is > 0) {
+            moe::PairProblem& q = P1.p[1];
+            MOE_TRY(make_map_gate_up_interleaved(&q.tw, W.w13s, 1, Is, c->H, "w13s"));
+            MOE_TRY(make_map(&q.tx, x, c->T, c->H, half, "x"));
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = c->H;
+            q.n_feat = Is;
+            q.out = at<void>(ws, L.ash);
+            q.ld_out = Is;
+            P1.n_problems = 2;
+        }
+        P1.status = status;
+    }
+    MOE_CUDA(moe::launch_pair_gemm(moe::EPI_SWIGLU, P1, sms, s), "gate/up pair GEMM launch");
+    if (ev_gemm2) MOE_CUDA(cudaEventRecord(ev_gemm2, s), "event record");
+
+    moe::PairParams P2;
+    memset(&P2, 0, sizeof(P2));
+    {
+        moe::PairProblem& p = P2.p[0];
+        MOE_TRY(make_map(&p.tw, W.w2, (size_t)c->E * c->H, c->I, 128, "w2"));
+        MOE_TRY(make_map(&p.tx, at<void>(ws, L.a), n, c->I, half, "expert activations"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->I;
+        p.n_feat = c->H;
+        p.out = y;
+        p.ld_out = c->H;
+        p.row_w = g.w_perm;
+        P2.n_problems = 1;
+        if (Is > 0) {
+            moe::PairProblem& q = P2.p[1];
+            MOE_TRY(make_map(&q.tw, W.w2s, c->H, Is, 128, "w2s"));
+            MOE_TRY(make_map(&q.tx, at<void>(ws, L.ash), c->T, Is, half, "shared activations"));
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = Is;
+            q.n_feat = c->H;
+            q.out = y_shared;
+            q.ld_out = c->H;
+            q.out_f32 = 1;
+            P2.n_problems = 2;
+        }
+        P2.status = status;
+    }
+    MOE_CUDA(moe::launch_pair_gemm(moe::EPI_SCALE, P2, sms, s), "down pair GEMM launch");
+    return MOE_OK;
+}
+
 moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t* offsets,
                             const int32_t* pos, const float* topk_w, const Weights& W, void* y,
                             void* y_shared, void* ws, cudaStream_t s, cudaEvent_t ev_mid,
@@ -274,6 +368,9 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
     int sms = 0;
     MOE_TRY(sm_count(&sms));
     int* status = at<int>(ws, L.status);
+    if (bn == moe::kPairTokens)
+        return run_expert_ffn_pairs(c, x, offsets, W, y, y_shared, ws, s, ev_gemm2, g, sms,
+                                    status);
 
     // gate/up GEMM + SwiGLU: routed experts, then the shared expert
     moe::GemmParams P1;
@@ -342,6 +439,7 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
             q.out = y_shared;
             q.ld_out = c->H;
             q.row_w = nullptr;
+            q.out_f32 = 1;
             P2.n_problems = 2;
         }
         P2.status = status;
@@ -355,7 +453,7 @@ moe_status_t run_combine(const moe_config_t* c, const void* y, const int32_t* po
     moe::CombineArgs a;
     a.y = static_cast<const uint16_t*>(y);
     a.pos = pos;
-    a.y_shared = static_cast<const uint16_t*>(y_shared);
+    a.y_shared = static_cast<const float*>(y_shared);
     a.out = static_cast<uint16_t*>(out);
     a.T = c->T;
     a.k = c->k;

@@ -253,14 +253,10 @@ __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
         }
     }
     if (a.y_shared) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.y_shared + (size_t)t * a.H) + c);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(p[i]);
-            acc[2 * i] += f.x;
-            acc[2 * i + 1] += f.y;
-        }
+        const float4* ys = reinterpret_cast<const float4*>(a.y_shared + (size_t)t * a.H) + 2 * c;
+        const float4 v0 = __ldg(ys), v1 = __ldg(ys + 1);
+        acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+        acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
     }
     uint4 o;
     __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);

@@ -293,12 +293,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 } else if (EPI == EPI_SCALE) {
                     tmem_wait_ld();
                     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+                    float* outf = reinterpret_cast<float*>(p.out);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         if (c0 + j < tl.nvalid && fok) {
                             const int row = tl.row0 + c0 + j;
                             const float wr = p.row_w ? __ldg(p.row_w + row) : 1.0f;
-                            out[(size_t)row * p.ld_out + f] = __float2bfloat16_rn(__uint_as_float(r[j]) * wr);
+                            const float v = __uint_as_float(r[j]) * wr;
+                            if (p.out_f32)
+                                outf[(size_t)row * p.ld_out + f] = v;
+                            else
+                                out[(size_t)row * p.ld_out + f] = __float2bfloat16_rn(v);
                         }
                     }
                 } else {

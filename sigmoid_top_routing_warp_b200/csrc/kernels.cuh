@@ -48,7 +48,7 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
 struct CombineArgs {
     const uint16_t* y;        // bf16 [T*k, H]
     const int32_t* pos;       // [T*k]
-    const uint16_t* y_shared; // bf16 [T, H] or null
+    const float* y_shared;    // fp32 [T, H] or null
     uint16_t* out;            // bf16 [T, H]
     int T, k, H;
 };
@@ -74,6 +74,7 @@ struct GemmProblem {
     void* out;                // [rows, ld_out] (fp32 for EPI_F32, bf16 otherwise)
     int ld_out;
     const float* row_w;       // EPI_SCALE: per-row factor, or null (1.0)
+    int out_f32;              // EPI_SCALE: store fp32 instead of bf16
 };
 
 struct GemmParams {
@@ -85,5 +86,37 @@ struct GemmParams {
 // bn: token tile (16, 64 or 128).  grid: persistent CTAs.
 cudaError_t launch_grouped_gemm(int epi, int bn, const GemmParams& params, int grid,
                                 cudaStream_t s);
+
+// ---------------------------------------------------------------- CTA-pair grouped GEMM
+// Prefill-sized version of the grouped GEMM: clusters of two CTAs run one
+// M = 256 MMA per K step (128 weight rows per CTA) over a 256-token tile
+// (128 token rows loaded per CTA).
+constexpr int kPairTokens = 256;
+
+struct PairProblem {
+    // EPI_SWIGLU: 5-D view {K, 8, 2, n_feat/8, n_exp} of the packed gate/up
+    // matrix [n_exp][2 n_feat][K] (box {64, 8, 2, 8, 1}: 64 features as
+    // 8-row gate / up blocks).  EPI_SCALE: 2-D [n_exp * n_feat, K], box {64, 128}.
+    CUtensorMap tw;
+    CUtensorMap tx;           // activations, bf16 2-D [rows, K], box {64, 128}
+    const int32_t* seg;       // [n_exp + 1] token-row offsets, or null: rows [0, n_rows)
+    const int32_t* tok_start; // [n_exp + 1] prefix of 256-token tiles, or null with seg
+    int n_exp;
+    int n_rows;
+    int K;                    // multiple of 64
+    int n_feat;               // output features per expert (multiple of 8)
+    void* out;                // bf16 [rows, ld_out] (fp32 if out_f32)
+    int ld_out;
+    const float* row_w;       // EPI_SCALE: per-row factor, or null (1.0)
+    int out_f32;              // EPI_SCALE: store fp32 instead of bf16
+};
+
+struct PairParams {
+    PairProblem p[2];
+    int n_problems;
+    int* status;
+};
+
+cudaError_t launch_pair_gemm(int epi, const PairParams& params, int grid, cudaStream_t s);
 
 }  // namespace moe

@@ -87,6 +87,9 @@ SMALL = [
     ("no_shared", 96, 512, 96, 8, 256, 0, 1, 1),
     ("k_equals_E", 40, 512, 32, 32, 128, 1, 1, 1),
     ("many_tokens", 1500, 512, 32, 4, 128, 1, 1, 1),
+    # prefill-sized: CTA-pair GEMMs with ragged tiles and H, I not multiples of 256
+    ("pair_ragged", 2000, 640, 32, 4, 384, 1, 1, 1),
+    ("pair_grouped", 4096, 1024, 64, 6, 256, 2, 4, 2),
 ]
 
 
@@ -126,7 +129,7 @@ def test_stage_entry_points_match_forward(B, W):
     pos = torch.empty((T * k,), dtype=torch.int32, device=dev)
     B.moe_permute(cfg, idx, offsets, rows, pos, ws2)
     y = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
-    ysh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ysh = torch.empty((T, H), dtype=torch.float32, device=dev)
     B.moe_expert_ffn(cfg, inp["x"], offsets, rows, pos, w, inp["w13"], inp["w2"], inp["w13s"],
                      inp["w2s"], y, ysh, ws2)
     out2 = torch.empty_like(out)
