@@ -142,6 +142,49 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ncu traffic
+
+KERNEL_SOURCES = {
+    "gate_up_decode": ["csrc/gemm.cu", "csrc/ptx.cuh", "csrc/kernels.cuh"],
+    "gate_up_prefill": ["csrc/gemm_pair.cu", "csrc/ptx.cuh", "csrc/kernels.cuh"],
+}
+
+
+def source_hash(kind):
+    import hashlib
+    m = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "sigmoid_top_routing_warp_b200", f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def profile_traffic(kind, algorithmic, workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summaries under profiles/, or None when there is none for this kernel or
+    the kernel's source changed since the counters were taken."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        fields = {}
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                line = line.strip()
+                if ":" in line and line.split(":", 1)[0] in (
+                        "kernel", "traffic_over_algorithmic", "traffic_bytes_per_launch",
+                        "source_hash", "workload"):
+                    k, v = line.split(":", 1)
+                    fields[k] = v.strip()
+        if fields.get("kernel") != kind or fields.get("source_hash") != source_hash(kind):
+            continue
+        if "traffic_bytes_per_launch" in fields and fields.get("workload") == workload:
+            return float(fields["traffic_bytes_per_launch"])
+        if "traffic_over_algorithmic" in fields:
+            return float(fields["traffic_over_algorithmic"]) * algorithmic
+    return None
+
+
 # ---------------------------------------------------------------- work model
 
 def layer_work(wl, touched: int):
@@ -357,17 +400,21 @@ def main():
     value = world * wl.T * K / (r["ms"] / 1e3)
     stage_names = r["B"].STAGE_NAMES
     g1_ms = float(r["stage_ms"][3])
+    pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0
+    kind = "gate_up_prefill" if pair else "gate_up_decode"
+    traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
     hbm_bound = work["bytes"] / (peaks["hbm_gbs"] * 1e9) >= work["flops"] / (
         peaks["bf16_tflops"] * 1e12)
     if hbm_bound:
         ach = work["g1_bytes"] / (g1_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": None}
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic}
     else:
         ach = work["g1_flops"] / (g1_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": None}
-    roof.update({"kernel": "grouped_gemm_kernel<SWIGLU> (gate/up GEMM + SwiGLU)",
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic}
+    roof.update({"kernel": ("pair_gemm_kernel<SWIGLU>" if pair else
+                            "grouped_gemm_kernel<SWIGLU,16>") + " (gate/up GEMM + SwiGLU)",
                  "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
                  "launch_ms": g1_ms, "peak_source": peak_src})
     layer_ms = r["ms"] / K
