@@ -199,6 +199,13 @@ moe_status_t sm_count(int* n) {
         if (st_ != MOE_OK) return st_;      \
     } while (0)
 
+// The token boxes of the CTA-pair kernels: 16, 32, 64 and 128 rows.
+moe_status_t make_pair_boxes(CUtensorMap* maps, const void* ptr, size_t rows, size_t cols,
+                             const char* what) {
+    for (int b = 0; b < moe::kPairBoxes; ++b) MOE_TRY(make_map(&maps[b], ptr, rows, cols, 16 << b, what));
+    return MOE_OK;
+}
+
 // ------------------------------------------------------------------ stages
 moe_status_t run_router_gemm(const moe_config_t* c, const void* x, const void* wg, float* logits,
                              int* status, cudaStream_t s) {
@@ -274,13 +281,12 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
     const Layout L = layout(c);
     const int n = c->T * c->k;
     const int Is = c->n_shared * c->I;
-    const int half = moe::kPairTokens / 2;
     moe::PairParams P1;
     memset(&P1, 0, sizeof(P1));
     {
         moe::PairProblem& p = P1.p[0];
         MOE_TRY(make_map_gate_up_interleaved(&p.tw, W.w13, c->E, c->I, c->H, "w13"));
-        MOE_TRY(make_map(&p.tx, g.x_perm, n, c->H, half, "gathered x"));
+        MOE_TRY(make_pair_boxes(p.tx, g.x_perm, n, c->H, "gathered x"));
         p.seg = offsets;
         p.tok_start = g.tok_start;
         p.n_exp = c->E;
@@ -292,7 +298,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
         if (Is > 0) {
             moe::PairProblem& q = P1.p[1];
             MOE_TRY(make_map_gate_up_interleaved(&q.tw, W.w13s, 1, Is, c->H, "w13s"));
-            MOE_TRY(make_map(&q.tx, x, c->T, c->H, half, "x"));
+            MOE_TRY(make_pair_boxes(q.tx, x, c->T, c->H, "x"));
             q.n_exp = 1;
             q.n_rows = c->T;
             q.K = c->H;
@@ -311,7 +317,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
     {
         moe::PairProblem& p = P2.p[0];
         MOE_TRY(make_map(&p.tw, W.w2, (size_t)c->E * c->H, c->I, 128, "w2"));
-        MOE_TRY(make_map(&p.tx, at<void>(ws, L.a), n, c->I, half, "expert activations"));
+        MOE_TRY(make_pair_boxes(p.tx, at<void>(ws, L.a), n, c->I, "expert activations"));
         p.seg = offsets;
         p.tok_start = g.tok_start;
         p.n_exp = c->E;
@@ -324,7 +330,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
         if (Is > 0) {
             moe::PairProblem& q = P2.p[1];
             MOE_TRY(make_map(&q.tw, W.w2s, c->H, Is, 128, "w2s"));
-            MOE_TRY(make_map(&q.tx, at<void>(ws, L.ash), c->T, Is, half, "shared activations"));
+            MOE_TRY(make_pair_boxes(q.tx, at<void>(ws, L.ash), c->T, Is, "shared activations"));
             q.n_exp = 1;
             q.n_rows = c->T;
             q.K = Is;

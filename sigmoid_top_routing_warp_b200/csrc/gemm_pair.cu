@@ -175,7 +175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     if (warp == 0 && lane == 0) {
         for (int pi = 0; pi < P.n_problems; ++pi) {
             tma_prefetch_desc(&P.p[pi].tw);
-            tma_prefetch_desc(&P.p[pi].tx);
+            for (int b = 0; b < kPairBoxes; ++b) tma_prefetch_desc(&P.p[pi].tx[b]);
         }
     }
     if (warp == 1) {
@@ -200,19 +200,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                 ptile_at<EPI>(P, t, tl);
                 const PairProblem& p = P.p[tl.prob];
                 const int nk = p.K / kPBK;
+                const int half = tile_n(tl.nvalid) >> 1;  // token rows this CTA feeds the MMA
+                int box = 0;
+                while ((16 << box) < half) ++box;
+                const uint32_t stage_bytes = kPWBytes + (16u << box) * kPBK * 2;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!wait_cl(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
                     uint8_t* st = smem + s * kPStage;
                     const uint32_t fb = full_leader + 8u * s;
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPStage);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
                     if (EPI == EPI_SWIGLU)
                         tma_load_5d_pair(st, &p.tw, fb, kb * kPBK, 0, 0, (tl.f0 + 64 * (int)cta) >> 3,
                                          tl.exp);
                     else
                         tma_load_2d_pair(st, &p.tw, fb, kb * kPBK,
                                          tl.exp * p.n_feat + tl.f0 + 128 * (int)cta);
-                    tma_load_2d_pair(st + kPWBytes, &p.tx, fb, kb * kPBK,
-                                     tl.row0 + (tile_n(tl.nvalid) >> 1) * (int)cta);
+                    tma_load_2d_pair(st + kPWBytes, &p.tx[box], fb, kb * kPBK,
+                                     tl.row0 + half * (int)cta);
                     issued |= 1u << s;
                     last_ph = (last_ph & ~(1u << s)) | (ph << s);
                     if (++s == kPStages) { s = 0; ph ^= 1; }

@@ -92,13 +92,16 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmParams& params, int g
 // M = 256 MMA per K step (128 weight rows per CTA) over a 256-token tile
 // (128 token rows loaded per CTA).
 constexpr int kPairTokens = 256;
+constexpr int kPairBoxes = 4;  // token boxes of 16, 32, 64, 128 rows per CTA
 
 struct PairProblem {
     // EPI_SWIGLU: 5-D view {K, 8, 2, n_feat/8, n_exp} of the packed gate/up
     // matrix [n_exp][2 n_feat][K] (box {64, 8, 2, 8, 1}: 64 features as
     // 8-row gate / up blocks).  EPI_SCALE: 2-D [n_exp * n_feat, K], box {64, 128}.
     CUtensorMap tw;
-    CUtensorMap tx;           // activations, bf16 2-D [rows, K], box {64, 128}
+    // activations, bf16 2-D [rows, K], box {64, 16 << i}: a tile loads only
+    // the rows it uses (its MMA width / 2 per CTA, rounded up to a box)
+    CUtensorMap tx[kPairBoxes];
     const int32_t* seg;       // [n_exp + 1] token-row offsets, or null: rows [0, n_rows)
     const int32_t* tok_start; // [n_exp + 1] prefix of 256-token tiles, or null with seg
     int n_exp;
