@@ -81,9 +81,23 @@ int expert_bn(const moe_config_t* c) {
 }
 int router_bn(const moe_config_t* c) { return c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128; }
 
+// K slices of the router GEMM: small batches have too few output tiles to
+// keep the GPU busy, so the K loop is split (the selection kernel sums the
+// slices in order).  The largest split of H/64 k-blocks into at most 16
+// slices that keeps the tile count within 148 CTAs.
+int router_split(const moe_config_t* c) {
+    const int bn = router_bn(c);
+    const int tiles = ((c->E + 127) / 128) * ((c->T + bn - 1) / bn);
+    const int nk = c->H / 64;
+    if (tiles >= 32) return 1;
+    for (int s = 16; s > 1; --s)
+        if (nk % s == 0 && tiles * s <= 148) return s;
+    return 1;
+}
+
 struct Layout {
-    size_t status, logits, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash, y,
-        ysh, total;
+    size_t status, logits, rpart, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash,
+        y, ysh, total;
 };
 
 Layout layout(const moe_config_t* c) {
@@ -98,6 +112,8 @@ Layout layout(const moe_config_t* c) {
     };
     L.status = take(256);
     L.logits = take(T * E * 4);
+    const int rs = router_split(c);
+    L.rpart = take(rs > 1 ? (size_t)rs * T * E * 4 : 0);
     L.idx = take(n * 4);
     L.w = take(n * 4);
     L.offsets = take((E + 1) * 4);
@@ -209,6 +225,7 @@ moe_status_t make_pair_boxes(CUtensorMap* maps, const void* ptr, size_t rows, si
 // ------------------------------------------------------------------ stages
 moe_status_t run_router_gemm(const moe_config_t* c, const void* x, const void* wg, float* logits,
                              int* status, cudaStream_t s) {
+    const int split = router_split(c);
     moe::GemmParams P;
     memset(&P, 0, sizeof(P));
     const int bn = router_bn(c);
@@ -225,20 +242,25 @@ moe_status_t run_router_gemm(const moe_config_t* c, const void* x, const void* w
     p.out = logits;
     p.ld_out = c->E;
     p.row_w = nullptr;
+    p.k_split = split;
+    p.split_stride = (long long)c->T * c->E;
     P.n_problems = 1;
     P.status = status;
     int sms = 0;
     MOE_TRY(sm_count(&sms));
-    const int tiles = ((c->E + 127) / 128) * ((c->T + bn - 1) / bn);
+    const int tiles = ((c->E + 127) / 128) * ((c->T + bn - 1) / bn) * split;
     const int grid = tiles < sms ? tiles : sms;
     MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_F32, bn, P, grid, s), "router GEMM launch");
     return MOE_OK;
 }
 
 moe_status_t run_select(const moe_config_t* c, const float* logits, const float* bias,
-                        int32_t* idx, float* w, cudaStream_t s) {
+                        int32_t* idx, float* w, cudaStream_t s, int n_split = 1,
+                        float* logits_out = nullptr) {
     moe::RouteArgs a;
     a.logits = logits;
+    a.n_split = n_split;
+    a.logits_out = logits_out;
     a.bias = bias;
     a.idx = idx;
     a.w = w;
@@ -525,8 +547,11 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_rou
     MOE_TRY(need(topk_w, "topk_w"));
     if (cfg->T == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    MOE_TRY(run_router_gemm(cfg, x, w_router, logits, at<int>(ws, layout(cfg).status), s));
-    return run_select(cfg, logits, bias, topk_idx, topk_w, s);
+    const Layout L = layout(cfg);
+    const int split = router_split(cfg);
+    float* gemm_out = split > 1 ? at<float>(ws, L.rpart) : logits;
+    MOE_TRY(run_router_gemm(cfg, x, w_router, gemm_out, at<int>(ws, L.status), s));
+    return run_select(cfg, gemm_out, bias, topk_idx, topk_w, s, split, logits);
 }
 
 moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
@@ -635,10 +660,12 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
     void* y = at<void>(ws, L.y);
     void* ysh = cfg->n_shared > 0 ? at<void>(ws, L.ysh) : nullptr;
 
+    const int split = router_split(cfg);
+    float* gemm_out = split > 1 ? at<float>(ws, L.rpart) : logits;
     MOE_TRY(mark(0));
-    MOE_TRY(run_router_gemm(cfg, x, w_router, logits, at<int>(ws, L.status), s));
+    MOE_TRY(run_router_gemm(cfg, x, w_router, gemm_out, at<int>(ws, L.status), s));
     MOE_TRY(mark(1));
-    MOE_TRY(run_select(cfg, logits, bias, idx, w, s));
+    MOE_TRY(run_select(cfg, gemm_out, bias, idx, w, s, split, logits));
     MOE_TRY(mark(2));
     MOE_TRY(run_permute(cfg, idx, offsets, at<int32_t>(ws, L.rows), pos, ws, s));
     Weights W{w13, w2, w13s, w2s};

@@ -65,12 +65,12 @@ struct Cfg {
 };
 
 struct Tile {
-    int prob, exp, row0, nvalid, f0;
+    int prob, exp, row0, nvalid, f0, kslice;
 };
 
 __device__ __forceinline__ int problem_tiles(const GemmProblem& p, int bn) {
     const int nf = (p.n_feat + 127) / 128;
-    if (p.seg == nullptr) return nf * ((p.n_rows + bn - 1) / bn);
+    if (p.seg == nullptr) return nf * ((p.n_rows + bn - 1) / bn) * max(p.k_split, 1);
     return nf * __ldg(p.tok_start + p.n_exp);
 }
 
@@ -87,6 +87,11 @@ __device__ __forceinline__ bool tile_at(const GemmParams& P, int bn, int t, Tile
         }
         const int nf = (p.n_feat + 127) / 128;
         int e = 0, first = 0, ntok, seg0, seg1;
+        o.kslice = 0;
+        if (p.seg == nullptr && p.k_split > 1) {
+            o.kslice = t % p.k_split;
+            t /= p.k_split;
+        }
         if (p.seg == nullptr) {
             ntok = (p.n_rows + bn - 1) / bn;
             seg0 = 0;
@@ -200,8 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 tile_at(P, BN, t, tl);
                 const GemmProblem& p = P.p[tl.prob];
                 const int wrow = tl.exp * p.w_rows + tl.f0;
-                const int nk = p.K / kBK;
-                for (int kb = 0; kb < nk; ++kb) {
+                const int nk = p.K / kBK / max(p.k_split, 1);
+                const int kb0 = tl.kslice * nk;
+                for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
                     uint8_t* st = smem + s * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 Tile tl;
                 tile_at(P, BN, t, tl);
-                const int nk = P.p[tl.prob].K / kBK;
+                const int nk = P.p[tl.prob].K / kBK / max(P.p[tl.prob].k_split, 1);
                 if (!wait_bar(&tempty[buf], aph ^ 1, abort_flag, P.status)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * C::ACC_COLS;
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                     }
                 } else {
                     tmem_wait_ld();
-                    float* out = reinterpret_cast<float*>(p.out);
+                    float* out = reinterpret_cast<float*>(p.out) + tl.kslice * p.split_stride;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (c0 + j < tl.nvalid && fok)

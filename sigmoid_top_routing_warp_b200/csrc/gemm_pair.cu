@@ -97,8 +97,11 @@ __device__ __forceinline__ bool ptile_at(const PairParams& P, int t, PTile& o) {
             seg0 = __ldg(p.seg + e);
             seg1 = __ldg(p.seg + e + 1);
         }
+        // feature tile innermost: the tiles running together share one token
+        // tile, and the expert's weights stay in L2 across its token tiles
         const int local = t - first;
-        const int ft = local / ntok, tt = local - ft * ntok;
+        const int tt = local / nf, ft = local - tt * nf;
+        (void)ntok;
         o.prob = pi;
         o.exp = e;
         o.f0 = ft * feat_tile<EPI>();

@@ -12,7 +12,9 @@ enum : int { DEV_STATUS_TIMEOUT = 1 };
 
 // ---------------------------------------------------------------- router
 struct RouteArgs {
-    const float* logits;  // [T, E]
+    const float* logits;  // [n_split, T, E]: logits, or K-slice partials summed in order
+    int n_split;          // 1: logits as given; > 1: sum the slices, write logits_out
+    float* logits_out;    // [T, E] summed logits (n_split > 1)
     const float* bias;    // [E]
     int32_t* idx;         // [T, k]
     float* w;             // [T, k]
@@ -75,6 +77,8 @@ struct GemmProblem {
     int ld_out;
     const float* row_w;       // EPI_SCALE: per-row factor, or null (1.0)
     int out_f32;              // EPI_SCALE: store fp32 instead of bf16
+    int k_split;              // EPI_F32: K slices (>= 1); slice s writes out + s * split_stride
+    long long split_stride;   // elements between the slices' outputs
 };
 
 struct GemmParams {

@@ -73,11 +73,29 @@ __global__ void __launch_bounds__(256) route_select_kernel(const RouteArgs a) {
     const int E = a.E, k = a.k;
     const int e0 = lane * VPL;
     const float* row = a.logits + (size_t)t * E + e0;
+    const size_t slice = (size_t)a.T * E;
+
+    float lg[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) lg[i] = __ldg(row + i);
+    if (a.n_split > 1) {
+        // K-slice partials of the router GEMM, summed in slice order (the
+        // loads of all slices are issued before the adds)
+        for (int sp = 1; sp < a.n_split; ++sp) {
+            float part[VPL];
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) part[i] = __ldg(row + sp * slice + i);
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) lg[i] = __fadd_rn(lg[i], part[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) a.logits_out[(size_t)t * E + e0 + i] = lg[i];
+    }
 
     float s[VPL], c[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const float l = __ldg(row + i);
+        const float l = lg[i];
         s[i] = dev_sigmoid(l);
         c[i] = __fadd_rn(s[i], __ldg(a.bias + e0 + i));  // bias steers the choice only
         if (isnan(c[i])) c[i] = -INFINITY;                // NaN ranks below numbers
