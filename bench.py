@@ -224,15 +224,18 @@ def profile_traffic(kind, algorithmic, workload):
 
 def layer_work(wl, touched: int):
     """Algorithmic FLOPs and HBM bytes of one layer call and of the gate/up
-    GEMM (the dominant kernel)."""
+    GEMM (the dominant kernel).  fp8 layers stream 1-byte weight codes (plus
+    one fp32 scale per 128x128 block) and 1-byte activation codes."""
     T, H, E, k, I, Is = wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is
-    el = 2  # bf16
+    el = 1 if wl.dtype == "fp8" else 2
+    sc = 4.0 / (128 * 128) if wl.dtype == "fp8" else 0.0   # scale bytes per weight
     flops = T * (2 * k * 3 * H * I + 2 * 3 * H * Is + 2 * H * E)
-    bytes_ = (touched * 3 * H * I + 3 * H * Is + E * H + 2 * T * H) * el
+    wbytes = (touched * 3 * H * I + 3 * H * Is) * (el + sc)
+    bytes_ = wbytes + E * H * 2 + 2 * T * H * 2
     g1_flops = 2 * T * k * 2 * I * H + 2 * T * 2 * Is * H
-    g1_bytes = (touched * 2 * I * H + 2 * Is * H      # weights streamed
-                + T * k * H + T * H                   # gathered + shared activations
-                + T * k * I + T * Is) * el            # SwiGLU outputs
+    g1_bytes = ((touched * 2 * I * H + 2 * Is * H) * (el + sc)   # weights streamed
+                + (T * k * H + T * H) * el                       # gathered + shared activations
+                + (T * k * I + T * Is) * el)                      # SwiGLU outputs
     return {"flops": flops, "bytes": bytes_, "g1_flops": g1_flops, "g1_bytes": g1_bytes}
 
 
@@ -253,14 +256,21 @@ def cfg_of(B, wl):
     return B.MoeConfig(T=wl.T, H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
                        n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
                        norm_topk_prob=wl.norm_topk_prob,
-                       routed_scaling_factor=wl.routed_scaling_factor)
+                       routed_scaling_factor=wl.routed_scaling_factor,
+                       dtype=B.MOE_DTYPE_FP8_E4M3_BLOCK128 if wl.dtype == "fp8" else
+                       B.MOE_DTYPE_BF16)
+
+
+def scales_of(inp):
+    return {k: inp[k] for k in ("w13_scale", "w2_scale", "w13s_scale", "w2s_scale") if k in inp}
 
 
 def launches_per_step(B, cfg):
     from sigmoid_top_routing_warp_b200 import build as _b  # noqa: F401
     permute = 1 if cfg.T * cfg.k <= 4096 else 3
-    # router GEMM, selection, permute, gather, gate/up GEMM, down GEMM, combine
-    return 2 + permute + 1 + 2 + 1
+    quant = 1 if cfg.dtype == B.MOE_DTYPE_FP8_E4M3_BLOCK128 else 0
+    # router GEMM, selection, permute, (fp8: quantise x), gather, gate/up GEMM, down GEMM, combine
+    return 2 + permute + quant + 1 + 2 + 1
 
 
 def run_ours(args, world, rank, local):
@@ -275,9 +285,11 @@ def run_ours(args, world, rank, local):
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    sc = scales_of(inp)
+
     def step(events=None):
         B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                      inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events)
+                      inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events, **sc)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -324,7 +336,7 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
         B.moe_forward(cfg, x_dev, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                      inp["w13s"], inp["w2s"], out, ws, stream=stream)
+                      inp["w13s"], inp["w2s"], out, ws, stream=stream, **sc)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -435,9 +447,15 @@ def main():
     value = world * wl.T * K / (r["ms"] / 1e3)
     stage_names = r["B"].STAGE_NAMES
     g1_ms = float(r["stage_ms"][3])
-    pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0
+    pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
     kind = "gate_up_prefill" if pair else "gate_up_decode"
     traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
+    fp8 = wl.dtype == "fp8"
+    if fp8:  # the fp8 tensor peak: the measured bf16 peaks x the nominal fp8/bf16 ratio 2
+        peaks = dict(peaks)
+        for key in ("bf16_tflops", "bf16_tflops_sustained"):
+            if key in peaks:
+                peaks[key] = 2.0 * peaks[key]
     hbm_bound = work["bytes"] / (peaks["hbm_gbs"] * 1e9) >= work["flops"] / (
         peaks["bf16_tflops"] * 1e12)
     if hbm_bound:
@@ -450,10 +468,12 @@ def main():
         ach = work["g1_flops"] / (g1_ms / 1e3) / 1e12
         pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
-                "frac": ach / pk, "traffic": traffic, "peak_kind": "bf16 sustained",
+                "frac": ach / pk, "traffic": traffic,
+                "peak_kind": "fp8 sustained (2x measured bf16)" if fp8 else "bf16 sustained",
                 "frac_of_burst_peak": ach / peaks["bf16_tflops"]}
-    roof.update({"kernel": ("pair_gemm_kernel<SWIGLU>" if pair else
-                            "grouped_gemm_kernel<SWIGLU,16>") + " (gate/up GEMM + SwiGLU)",
+    kname = ("fp8_gemm_kernel<SWIGLU>" if fp8 else "pair_gemm_kernel<SWIGLU>" if pair else
+             "grouped_gemm_kernel<SWIGLU,16>")
+    roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
                  "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
                  "launch_ms": g1_ms, "peak_source": peak_src})
     layer_ms = r["ms"] / K
@@ -468,7 +488,8 @@ def main():
     layer["frac_of_roofline"] = layer["t_roof_ms"] / layer_ms
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": layer_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
                        "I": wl.I, "n_shared": wl.n_shared, "n_group": wl.n_group,
                        "topk_group": wl.topk_group, "experts_touched": r["touched"],

@@ -67,7 +67,11 @@ typedef enum {
 } moe_status_t;
 
 typedef enum {
-    MOE_DTYPE_BF16 = 0 /* bf16 activations and weights, fp32 accumulation */
+    MOE_DTYPE_BF16 = 0,              /* bf16 activations and weights, fp32 accumulation */
+    MOE_DTYPE_FP8_E4M3_BLOCK128 = 1  /* expert weights e4m3 (OCP FP8, 1 byte) with one fp32
+                                        scale per 128 x 128 block; expert-GEMM activations
+                                        quantised to e4m3 per row and 128 columns
+                                        (moe_quantize_act); router stays bf16           */
 } moe_dtype_t;
 
 /* Layer description.  Field names follow the Dots1 / DeepSeek-V3 config:
@@ -180,14 +184,29 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_id
  *   y_shared fp32 [T, H] out  SwiGLU_shared(x) (may be NULL iff n_shared == 0);
  *            kept in fp32 because, with weight 1, it is the largest term of
  *            the combine and its rounding would dominate the output error
- * The *_scale arguments are reserved for block-scaled weights and must be
- * NULL for MOE_DTYPE_BF16.                                                  */
+ * For MOE_DTYPE_FP8_E4M3_BLOCK128 the four weight matrices hold e4m3 codes
+ * (same shapes, 1 byte each) and the *_scale arguments their fp32 block
+ * scales, row-major over 128 x 128 blocks:
+ *   w13_scale [E, 2I/128, H/128], w2_scale [E, H/128, I/128],
+ *   w13s_scale [2Is/128, H/128], w2s_scale [H/128, Is/128];
+ * weight value = code * scale of its block.  For MOE_DTYPE_BF16 the *_scale
+ * arguments must be NULL.                                                   */
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_t* offsets,
                             const int32_t* rows, const int32_t* pos, const float* topk_w,
                             const void* w13, const float* w13_scale, const void* w2,
                             const float* w2_scale, const void* w13s, const float* w13s_scale,
                             const void* w2s, const float* w2s_scale, void* y, void* y_shared,
                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Activation quantisation, step a0 of the FP8 layer (FP8 deployment:
+ * mlqm.cn 部署实战; the recipe is this library's, see moe_dtype_t): per row
+ * and 128 columns, scale = amax / 448 (1 for an all-zero block) and
+ * code = e4m3(x / scale), round to nearest even, saturating to +-448; both
+ * in correctly rounded binary32.
+ *   x bf16 [rows, cols] (cols a multiple of 128), q e4m3 codes [rows, cols]
+ *   out, scale fp32 [rows, cols/128] out.  No workspace.                    */
+moe_status_t moe_quantize_act(const void* x, int32_t rows, int32_t cols, uint8_t* q, float* scale,
+                              moe_stream_t stream);
 
 /* Combine: step a9 (Deep Dive §3.3 "Weighted sum" then shared "add").
  * out_t = sum_{j=0..k-1} y[pos[t*k + j]] + y_shared_t, summed in fp32 in

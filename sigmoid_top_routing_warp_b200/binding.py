@@ -22,6 +22,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
     MOE_ERR_TIMEOUT = range(6)
 MOE_DTYPE_BF16 = 0
+MOE_DTYPE_FP8_E4M3_BLOCK128 = 1
 MOE_NUM_STAGES = 6
 STAGE_NAMES = ("router_gemm", "router_select", "dispatch", "gate_up_swiglu", "down_weighted",
                "combine")
@@ -31,7 +32,8 @@ WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "p
 # Every symbol include/moe.h declares.
 EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
-            "moe_forward", "moe_check_device_status", "moe_permute_noalloc")
+            "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
+            "moe_quantize_act")
 
 
 class MoeConfigC(ctypes.Structure):
@@ -98,6 +100,8 @@ _lib.moe_forward.restype = ctypes.c_int
 _lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
 _lib.moe_permute_noalloc.restype = ctypes.c_int
 _lib.moe_permute_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P]
+_lib.moe_quantize_act.restype = ctypes.c_int
+_lib.moe_quantize_act.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -207,6 +211,13 @@ def moe_forward(cfg, x, w_router, bias, w13, w2, w13s, w2s, out, ws, stream=None
                             _ptr(w13_scale), _ptr(w2), _ptr(w2_scale), _ptr(w13s),
                             _ptr(w13s_scale), _ptr(w2s), _ptr(w2s_scale), _ptr(out), _ptr(ws),
                             ws.numel(), ev, _stream(stream)), "moe_forward")
+
+
+def moe_quantize_act(x, q, scale, stream=None):
+    """Step a0 of the FP8 layer: e4m3 codes and per-(row, 128-column) scales."""
+    rows, cols = x.shape
+    _check(_lib.moe_quantize_act(_ptr(x), rows, cols, _ptr(q), _ptr(scale), _stream(stream)),
+           "moe_quantize_act")
 
 
 def moe_check_device_status(ws, stream=None):

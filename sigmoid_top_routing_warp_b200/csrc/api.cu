@@ -41,7 +41,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 moe_status_t check_config(const moe_config_t* c) {
     if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
     if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d must be >= 0", c->T);
-    if (c->dtype != MOE_DTYPE_BF16)
+    if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_FP8_E4M3_BLOCK128)
         return fail(MOE_ERR_UNSUPPORTED, "dtype %d not supported", c->dtype);
     if (c->H <= 0 || c->H % 128)
         return fail(MOE_ERR_UNSUPPORTED, "H=%d must be a positive multiple of 128", c->H);
@@ -79,6 +79,15 @@ int expert_bn(const moe_config_t* c) {
     const double avg = c->E ? (double)c->T * c->k / c->E : 0.0;
     return avg <= 24.0 ? 16 : avg <= 96.0 ? 64 : moe::kPairTokens;
 }
+inline bool is_fp8(const moe_config_t* c) { return c->dtype == MOE_DTYPE_FP8_E4M3_BLOCK128; }
+
+// Token tile of the FP8 expert GEMMs (register accumulators: 16, 32 or 64
+// tokens; 64-token tiles use eight epilogue warps).
+int fp8_bn(const moe_config_t* c) {
+    const double avg = c->E ? (double)c->T * c->k / c->E : 0.0;
+    return avg <= 24.0 ? 16 : avg <= 48.0 ? 32 : 64;
+}
+
 int router_bn(const moe_config_t* c) { return c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128; }
 
 // K slices of the router GEMM: small batches have too few output tiles to
@@ -97,7 +106,7 @@ int router_split(const moe_config_t* c) {
 
 struct Layout {
     size_t status, logits, rpart, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash,
-        y, ysh, total;
+        y, ysh, xq, sx, xpq, sxp, aq, sa, ashq, sash, total;
 };
 
 Layout layout(const moe_config_t* c) {
@@ -127,6 +136,15 @@ Layout layout(const moe_config_t* c) {
     L.ash = take(T * Is * 2);
     L.y = take(n * H * 2);
     L.ysh = take(T * H * 4);
+    const bool q = is_fp8(c);
+    L.xq = take(q ? T * H : 0);
+    L.sx = take(q ? T * (H / 128) * 4 : 0);
+    L.xpq = take(q ? n * H : 0);
+    L.sxp = take(q ? n * (H / 128) * 4 : 0);
+    L.aq = take(q ? n * I : 0);
+    L.sa = take(q ? n * (I / 128) * 4 : 0);
+    L.ashq = take(q ? T * Is : 0);
+    L.sash = take(q ? T * (Is / 128) * 4 : 0);
     L.total = off;
     return L;
 }
@@ -215,6 +233,24 @@ moe_status_t sm_count(int* n) {
         if (st_ != MOE_OK) return st_;      \
     } while (0)
 
+// e4m3 codes (1 byte) row-major [rows, cols] as a 2-D tensor, box {128
+// columns, box_rows}, 128-byte swizzle (K-major rows of 128 bytes).
+moe_status_t make_map_u8(CUtensorMap* m, const void* ptr, size_t rows, size_t cols, int box_rows,
+                         const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
+
 // The token boxes of the CTA-pair kernels: 16, 32, 64 and 128 rows.
 moe_status_t make_pair_boxes(CUtensorMap* maps, const void* ptr, size_t rows, size_t cols,
                              const char* what) {
@@ -293,7 +329,125 @@ moe_status_t run_permute(const moe_config_t* c, const int32_t* idx, int32_t* off
 
 struct Weights {
     const void *w13, *w2, *w13s, *w2s;
+    const float *s13, *s2, *s13s, *s2s;  // fp8 block scales (null for bf16)
 };
+
+// FP8 layer: a0 quantisation of x, gather of codes and scales, then both
+// expert GEMMs on e4m3 operands with scale promotion (gemm_fp8.cu).
+moe_status_t run_expert_ffn_fp8(const moe_config_t* c, const void* x, const int32_t* offsets,
+                                const int32_t* pos, const float* topk_w, const Weights& W,
+                                void* y, void* y_shared, void* ws, cudaStream_t s,
+                                cudaEvent_t ev_mid, cudaEvent_t ev_gemm2) {
+    const Layout L = layout(c);
+    const int bn = fp8_bn(c);
+    const int n = c->T * c->k;
+    const int Is = c->n_shared * c->I;
+    moe::QuantArgs qa;
+    qa.x = static_cast<const uint16_t*>(x);
+    qa.q = at<uint8_t>(ws, L.xq);
+    qa.scale = at<float>(ws, L.sx);
+    qa.rows = c->T;
+    qa.cols = c->H;
+    MOE_CUDA(moe::launch_quant_act(qa, s), "activation quantisation launch");
+    moe::GatherQArgs g;
+    g.xq = qa.q;
+    g.sx = qa.scale;
+    g.pos = pos;
+    g.topk_w = topk_w;
+    g.offsets = offsets;
+    g.xq_perm = at<uint8_t>(ws, L.xpq);
+    g.sx_perm = at<float>(ws, L.sxp);
+    g.w_perm = at<float>(ws, L.wperm);
+    g.tok_start = at<int32_t>(ws, L.tokstart);
+    g.T = c->T;
+    g.k = c->k;
+    g.H = c->H;
+    g.E = c->E;
+    g.bn = bn;
+    MOE_CUDA(moe::launch_gather_q(g, s), "fp8 gather launch");
+    if (ev_mid) MOE_CUDA(cudaEventRecord(ev_mid, s), "event record");
+    int sms = 0;
+    MOE_TRY(sm_count(&sms));
+    int* status = at<int>(ws, L.status);
+
+    moe::GemmParams P1;
+    memset(&P1, 0, sizeof(P1));
+    {
+        moe::GemmProblem& p = P1.p[0];
+        MOE_TRY(make_map_u8(&p.tw, W.w13, (size_t)c->E * 2 * c->I, c->H, 128, "w13"));
+        MOE_TRY(make_map_u8(&p.tx, g.xq_perm, n, c->H, bn, "gathered x codes"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->H;
+        p.n_feat = c->I;
+        p.w_rows = 2 * c->I;
+        p.ld_out = c->I;
+        p.w_scale = W.s13;
+        p.x_scale = g.sx_perm;
+        p.out_q = at<uint8_t>(ws, L.aq);
+        p.out_scale = at<float>(ws, L.sa);
+        P1.n_problems = 1;
+        if (Is > 0) {
+            moe::GemmProblem& q = P1.p[1];
+            MOE_TRY(make_map_u8(&q.tw, W.w13s, (size_t)2 * Is, c->H, 128, "w13s"));
+            MOE_TRY(make_map_u8(&q.tx, qa.q, c->T, c->H, bn, "x codes"));
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = c->H;
+            q.n_feat = Is;
+            q.w_rows = 2 * Is;
+            q.ld_out = Is;
+            q.w_scale = W.s13s;
+            q.x_scale = qa.scale;
+            q.out_q = at<uint8_t>(ws, L.ashq);
+            q.out_scale = at<float>(ws, L.sash);
+            P1.n_problems = 2;
+        }
+        P1.status = status;
+    }
+    MOE_CUDA(moe::launch_fp8_gemm(moe::EPI_SWIGLU, bn, P1, sms, s), "fp8 gate/up GEMM launch");
+    if (ev_gemm2) MOE_CUDA(cudaEventRecord(ev_gemm2, s), "event record");
+
+    moe::GemmParams P2;
+    memset(&P2, 0, sizeof(P2));
+    {
+        moe::GemmProblem& p = P2.p[0];
+        MOE_TRY(make_map_u8(&p.tw, W.w2, (size_t)c->E * c->H, c->I, 128, "w2"));
+        MOE_TRY(make_map_u8(&p.tx, at<void>(ws, L.aq), n, c->I, bn, "expert activation codes"));
+        p.seg = offsets;
+        p.tok_start = g.tok_start;
+        p.n_exp = c->E;
+        p.K = c->I;
+        p.n_feat = c->H;
+        p.w_rows = c->H;
+        p.out = y;
+        p.ld_out = c->H;
+        p.row_w = g.w_perm;
+        p.w_scale = W.s2;
+        p.x_scale = at<float>(ws, L.sa);
+        P2.n_problems = 1;
+        if (Is > 0) {
+            moe::GemmProblem& q = P2.p[1];
+            MOE_TRY(make_map_u8(&q.tw, W.w2s, c->H, Is, 128, "w2s"));
+            MOE_TRY(make_map_u8(&q.tx, at<void>(ws, L.ashq), c->T, Is, bn, "shared activation codes"));
+            q.n_exp = 1;
+            q.n_rows = c->T;
+            q.K = Is;
+            q.n_feat = c->H;
+            q.w_rows = c->H;
+            q.out = y_shared;
+            q.ld_out = c->H;
+            q.out_f32 = 1;
+            q.w_scale = W.s2s;
+            q.x_scale = at<float>(ws, L.sash);
+            P2.n_problems = 2;
+        }
+        P2.status = status;
+    }
+    MOE_CUDA(moe::launch_fp8_gemm(moe::EPI_SCALE, bn, P2, sms, s), "fp8 down GEMM launch");
+    return MOE_OK;
+}
 
 // Prefill-sized batches: both expert GEMMs on CTA pairs (256 x 256 tiles).
 moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const int32_t* offsets,
@@ -372,6 +526,8 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
                             const int32_t* pos, const float* topk_w, const Weights& W, void* y,
                             void* y_shared, void* ws, cudaStream_t s, cudaEvent_t ev_mid,
                             cudaEvent_t ev_gemm2) {
+    if (is_fp8(c))
+        return run_expert_ffn_fp8(c, x, offsets, pos, topk_w, W, y, y_shared, ws, s, ev_mid, ev_gemm2);
     const Layout L = layout(c);
     const int bn = expert_bn(c);
     const int n = c->T * c->k;
@@ -499,9 +655,16 @@ moe_status_t need16(const void* p, const char* name) {
     return aligned16(p) ? MOE_OK : fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
 }
 
-moe_status_t check_scales(const float* a, const float* b, const float* c2, const float* d) {
-    if (a || b || c2 || d)
-        return fail(MOE_ERR_INVALID_ARG, "weight scales must be NULL for bf16 weights");
+moe_status_t check_scales(const moe_config_t* cfg, const float* a, const float* b, const float* c2,
+                          const float* d) {
+    if (!is_fp8(cfg)) {
+        if (a || b || c2 || d)
+            return fail(MOE_ERR_INVALID_ARG, "weight scales must be NULL for bf16 weights");
+        return MOE_OK;
+    }
+    if (!a || !b) return fail(MOE_ERR_INVALID_ARG, "fp8 weights need w13_scale and w2_scale");
+    if (cfg->n_shared > 0 && (!c2 || !d))
+        return fail(MOE_ERR_INVALID_ARG, "fp8 shared weights need w13s_scale and w2s_scale");
     return MOE_OK;
 }
 
@@ -589,7 +752,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_
     g_err[0] = 0;
     MOE_TRY(check_config(cfg));
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    MOE_TRY(check_scales(w13_scale, w2_scale, w13s_scale, w2s_scale));
+    MOE_TRY(check_scales(cfg, w13_scale, w2_scale, w13s_scale, w2s_scale));
     MOE_TRY(need16(x, "x"));
     MOE_TRY(need(offsets, "offsets"));
     MOE_TRY(need(rows, "rows"));
@@ -604,7 +767,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_
         MOE_TRY(need16(y_shared, "y_shared"));
     }
     if (cfg->T == 0) return MOE_OK;
-    Weights W{w13, w2, w13s, w2s};
+    Weights W{w13, w2, w13s, w2s, w13_scale, w2_scale, w13s_scale, w2s_scale};
     return run_expert_ffn(cfg, x, offsets, pos, topk_w, W, y, y_shared, ws,
                           static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
@@ -631,7 +794,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
     g_err[0] = 0;
     MOE_TRY(check_config(cfg));
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    MOE_TRY(check_scales(w13_scale, w2_scale, w13s_scale, w2s_scale));
+    MOE_TRY(check_scales(cfg, w13_scale, w2_scale, w13s_scale, w2s_scale));
     MOE_TRY(need16(x, "x"));
     MOE_TRY(need16(w_router, "w_router"));
     MOE_TRY(need(bias, "bias"));
@@ -668,11 +831,31 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
     MOE_TRY(run_select(cfg, gemm_out, bias, idx, w, s, split, logits));
     MOE_TRY(mark(2));
     MOE_TRY(run_permute(cfg, idx, offsets, at<int32_t>(ws, L.rows), pos, ws, s));
-    Weights W{w13, w2, w13s, w2s};
+    Weights W{w13, w2, w13s, w2s, w13_scale, w2_scale, w13s_scale, w2s_scale};
     MOE_TRY(run_expert_ffn(cfg, x, offsets, pos, w, W, y, ysh, ws, s, ev[3], ev[4]));
     MOE_TRY(mark(5));
     MOE_TRY(run_combine(cfg, y, pos, ysh, out, s));
     return mark(6);
+}
+
+moe_status_t moe_quantize_act(const void* x, int32_t rows, int32_t cols, uint8_t* q, float* scale,
+                              moe_stream_t stream) {
+    g_err[0] = 0;
+    if (rows < 0 || cols <= 0 || cols % 128)
+        return fail(MOE_ERR_INVALID_ARG, "rows=%d cols=%d: cols must be a positive multiple of 128",
+                    rows, cols);
+    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need16(q, "q"));
+    MOE_TRY(need(scale, "scale"));
+    if (rows == 0) return MOE_OK;
+    moe::QuantArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.q = q;
+    a.scale = scale;
+    a.rows = rows;
+    a.cols = cols;
+    MOE_CUDA(moe::launch_quant_act(a, static_cast<cudaStream_t>(stream)), "quantisation launch");
+    return MOE_OK;
 }
 
 moe_status_t moe_check_device_status(void* ws, moe_stream_t stream) {

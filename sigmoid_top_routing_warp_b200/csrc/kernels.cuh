@@ -56,6 +56,33 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
+// ---------------------------------------------------------------- FP8 (e4m3, 128-blocks)
+// Activation quantisation: per row, per 128 columns, scale = amax / 448,
+// codes = RNE-satfinite e4m3(x / scale); an all-zero block gets scale 1.
+struct QuantArgs {
+    const uint16_t* x;   // bf16 [rows, cols]
+    uint8_t* q;          // e4m3 [rows, cols]
+    float* scale;        // [rows, cols / 128]
+    int rows, cols;      // cols multiple of 128
+};
+cudaError_t launch_quant_act(const QuantArgs& a, cudaStream_t s);
+
+// Row gather of e4m3 codes and their scales, plus the routing weight per
+// sorted row and the token-tile prefix (as launch_gather).
+struct GatherQArgs {
+    const uint8_t* xq;        // [T, H]
+    const float* sx;          // [T, H/128]
+    const int32_t* pos;       // [T*k]
+    const float* topk_w;      // [T*k]
+    const int32_t* offsets;   // [E + 1]
+    uint8_t* xq_perm;         // [T*k, H]
+    float* sx_perm;           // [T*k, H/128]
+    float* w_perm;            // [T*k]
+    int32_t* tok_start;       // [E + 1]
+    int T, k, H, E, bn;
+};
+cudaError_t launch_gather_q(const GatherQArgs& a, cudaStream_t s);
+
 // ---------------------------------------------------------------- grouped GEMM
 enum Epilogue : int { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_SCALE = 2 };
 
@@ -79,6 +106,11 @@ struct GemmProblem {
     int out_f32;              // EPI_SCALE: store fp32 instead of bf16
     int k_split;              // EPI_F32: K slices (>= 1); slice s writes out + s * split_stride
     long long split_stride;   // elements between the slices' outputs
+    // FP8 (e4m3 operands with fp32 scales per 128-block, see gemm_fp8.cu):
+    const float* w_scale;     // [n_exp][w_rows/128][K/128] weight block scales
+    const float* x_scale;     // [rows][K/128] activation scales
+    uint8_t* out_q;           // EPI_SWIGLU: e4m3 codes [rows, ld_out]
+    float* out_scale;         // EPI_SWIGLU: scales [rows, ld_out/128]
 };
 
 struct GemmParams {
@@ -125,5 +157,9 @@ struct PairParams {
 };
 
 cudaError_t launch_pair_gemm(int epi, const PairParams& params, int grid, cudaStream_t s);
+
+// FP8 grouped GEMM (single CTA, weights as the M operand): EPI_SWIGLU
+// (writes e4m3 codes + scales of A) or EPI_SCALE (bf16 / fp32 out).  bn 16 or 32.
+cudaError_t launch_fp8_gemm(int epi, int bn, const GemmParams& params, int grid, cudaStream_t s);
 
 }  // namespace moe

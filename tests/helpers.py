@@ -20,12 +20,27 @@ def u16(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
+REL_L2_FP8 = 3e-2
+
+
+def is_fp8(c) -> bool:
+    return getattr(c, "dtype", 0) in (1, "fp8")
+
+
 def oracle_cfg(wl_or_cfg, T=None) -> O.Config:
     c = wl_or_cfg
     return O.Config(T=c.T if T is None else T, H=c.H, E=c.E, k=c.k, I=c.I, n_shared=c.n_shared,
                     n_group=c.n_group, topk_group=c.topk_group, group_topn=c.group_topn,
                     norm_topk_prob=c.norm_topk_prob,
-                    routed_scaling_factor=c.routed_scaling_factor)
+                    routed_scaling_factor=c.routed_scaling_factor, fp8=is_fp8(c))
+
+
+def u8(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().numpy().astype(np.uint8)
+
+
+def f32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().float().numpy()
 
 
 def oracle_layer_on_tokens(cfg, inp, idx: np.ndarray, w: np.ndarray, tokens) -> np.ndarray:
@@ -41,9 +56,22 @@ def oracle_layer_on_tokens(cfg, inp, idx: np.ndarray, w: np.ndarray, tokens) -> 
     oc.E = int(used.size)
     oc.k = cfg.k
     x = u16(inp["x"][torch.as_tensor(tokens, device=inp["x"].device)])
+    if oc.fp8:
+        return O.layer(oc, x, remap[sub_idx].astype(np.int32), w[tokens],
+                       u8(inp["w13"][sel]), u8(inp["w2"][sel]), u8(inp["w13s"]), u8(inp["w2s"]),
+                       w13_scale=f32(inp["w13_scale"][sel]), w2_scale=f32(inp["w2_scale"][sel]),
+                       w13s_scale=f32(inp["w13s_scale"]), w2s_scale=f32(inp["w2s_scale"]))
     return O.layer(oc, x, remap[sub_idx].astype(np.int32), w[tokens],
                    u16(inp["w13"][sel]), u16(inp["w2"][sel]), u16(inp["w13s"]),
                    u16(inp["w2s"]))
+
+
+def assert_close_fp8(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert rel <= REL_L2_FP8, "%s: rel-L2 %.3e > %.0e" % (what, rel, REL_L2_FP8)
+    return rel
 
 
 def assert_close_bf16(got: np.ndarray, ref: np.ndarray, what: str = ""):
@@ -57,3 +85,16 @@ def assert_close_bf16(got: np.ndarray, ref: np.ndarray, what: str = ""):
     assert mx <= MAX_ABS_RMS_BF16 * rms, "%s: max-abs %.3e > %.0e * rms %.3e" % (
         what, mx, MAX_ABS_RMS_BF16, rms)
     return rel, mx / max(rms, 1e-30)
+
+
+def check_routing_fn(B, cfg, ws, inp):
+    """Routing of a forward pass against the oracle fed the GPU's fp32 logits:
+    indices and weights must match bit for bit.  Returns (logits, idx, w,
+    near-tie count)."""
+    L = B.ws_view(ws, cfg, "logits").cpu().numpy()
+    idx = B.ws_view(ws, cfg, "topk_idx").cpu().numpy()
+    w = B.ws_view(ws, cfg, "topk_w").cpu().numpy()
+    oidx, ow, gap = O.route(oracle_cfg(cfg), L, inp["bias"].cpu().numpy())
+    assert (idx == oidx).all(), "routing indices differ on %d tokens" % (idx != oidx).any(1).sum()
+    assert (w.view(np.uint32) == ow.view(np.uint32)).all(), "routing weights differ"
+    return L, idx, w, int((gap < NEAR_TIE).sum())
