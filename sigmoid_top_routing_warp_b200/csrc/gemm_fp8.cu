@@ -209,38 +209,60 @@ __global__ void __launch_bounds__(QCfg<EPI, BN>::THREADS, 1)
             for (int w = 0; w < C::NW; ++w)
 #pragma unroll
                 for (int j = 0; j < C::CW; ++j) acc[w][j] = 0.0f;
-            for (int kb = 0; kb < nk; ++kb) {
-                if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t r[C::NW][C::CW];
-                const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + pb * C::PART_COLS + cb;
+            // Scales, fetched SC K blocks at a time one chunk ahead so that their
+            // global-load latency overlaps the promotion of the previous chunk:
+            // weight blocks (one per 128-row tile) and lane j's token cb + j.
+            constexpr int SC = C::EW == 8 ? 2 : 4;  // 8-warp variants have fewer registers
+            const int jl = cb + lane;
+            const bool jv = lane < C::CW && jl < tl.nvalid;
+            const float* xs = p.x_scale + (size_t)(tl.row0 + (jv ? jl : 0)) * kbs;
+            const float* wsp[C::NW];
 #pragma unroll
-                for (int w = 0; w < C::NW; ++w)
+            for (int w = 0; w < C::NW; ++w)
+                wsp[w] = p.w_scale + (size_t)((tl.exp * p.w_rows + tl.f0 + w * p.n_feat) / 128) * kbs;
+            float nx[SC], nw[C::NW][SC];
 #pragma unroll
-                    for (int c0 = 0; c0 < C::CW; c0 += 16)
-                        tmem_ld_16(tb + w * BN + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[w][c0]));
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pempty[pb]);
-                if (++pb == C::NP) { pb = 0; pph ^= 1; }
-                // scales: weight block (one per 128-row tile) x activation (per token)
-                float sw[C::NW];
+            for (int i = 0; i < SC; ++i) {
+                nx[i] = (jv && i < nk) ? __ldg(xs + i) : 0.0f;
 #pragma unroll
-                for (int w = 0; w < C::NW; ++w) {
-                    const int wr = tl.exp * p.w_rows + tl.f0 + w * p.n_feat;  // first weight row
-                    sw[w] = __ldg(p.w_scale + (size_t)(wr / 128) * kbs + kb);
+                for (int w = 0; w < C::NW; ++w) nw[w][i] = i < nk ? __ldg(wsp[w] + i) : 0.0f;
+            }
+            for (int k0 = 0; k0 < nk && ok; k0 += SC) {
+                float cx[SC], cw[C::NW][SC];
+#pragma unroll
+                for (int i = 0; i < SC; ++i) {
+                    cx[i] = nx[i];
+#pragma unroll
+                    for (int w = 0; w < C::NW; ++w) cw[w][i] = nw[w][i];
+                    const int kn = k0 + SC + i;
+                    nx[i] = (jv && kn < nk) ? __ldg(xs + kn) : 0.0f;
+#pragma unroll
+                    for (int w = 0; w < C::NW; ++w) nw[w][i] = kn < nk ? __ldg(wsp[w] + kn) : 0.0f;
                 }
-                // CW <= 32: lane j holds the activation scale of column cb + j
-                const int jl = cb + lane;
-                const float sx_l = (lane < C::CW && jl < tl.nvalid)
-                                       ? __ldg(p.x_scale + (size_t)(tl.row0 + jl) * kbs + kb) : 0.0f;
 #pragma unroll
-                for (int j = 0; j < C::CW; ++j) {
-                    const float sxj = __shfl_sync(0xffffffffu, sx_l, j);
+                for (int i = 0; i < SC; ++i) {
+                    if (k0 + i >= nk) break;
+                    if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t r[C::NW][C::CW];
+                    const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + pb * C::PART_COLS + cb;
 #pragma unroll
                     for (int w = 0; w < C::NW; ++w)
-                        acc[w][j] = fmaf(sw[w] * sxj, __uint_as_float(r[w][j]), acc[w][j]);
+#pragma unroll
+                        for (int c0 = 0; c0 < C::CW; c0 += 16)
+                            tmem_ld_16(tb + w * BN + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[w][c0]));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pempty[pb]);
+                    if (++pb == C::NP) { pb = 0; pph ^= 1; }
+#pragma unroll
+                    for (int j = 0; j < C::CW; ++j) {
+                        const float sxj = __shfl_sync(0xffffffffu, cx[i], j);
+#pragma unroll
+                        for (int w = 0; w < C::NW; ++w)
+                            acc[w][j] = fmaf(cw[w][i] * sxj, __uint_as_float(r[w][j]), acc[w][j]);
+                    }
                 }
             }
             if (!ok) break;
