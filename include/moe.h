@@ -88,7 +88,7 @@ typedef enum {
  *   norm_topk_prob         non-zero: divide weights by their sum
  *   routed_scaling_factor  multiplies the routed weights (1.0)
  *   dtype                  moe_dtype_t
- *   flags                  0 (reserved)                                     */
+ *   flags                  0, or MOE_FLAG_TEST_STALL (tests only)           */
 typedef struct {
     int32_t T, H, E, k, I, n_shared;
     int32_t n_group, topk_group, group_topn;
@@ -97,6 +97,13 @@ typedef struct {
     int32_t dtype;
     uint32_t flags;
 } moe_config_t;
+
+/* Test of the device-side failure path, never set in normal use: the first
+ * CTA of the router GEMM leaves its first pipeline stage unfilled, so its
+ * bounded wait runs out (about one second), the kernel records a timeout in
+ * the workspace status word and returns; moe_check_device_status then
+ * reports MOE_ERR_TIMEOUT and the CUDA context stays usable. */
+#define MOE_FLAG_TEST_STALL 0x1u
 
 /* A cudaStream_t. */
 typedef void* moe_stream_t;

@@ -24,6 +24,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3_BLOCK128 = 1
 MOE_NUM_STAGES = 6
+MOE_FLAG_TEST_STALL = 0x1
 STAGE_NAMES = ("router_gemm", "router_select", "dispatch", "gate_up_swiglu", "down_weighted",
                "combine")
 WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "pos": 5,

@@ -52,6 +52,8 @@ moe_status_t check_config(const moe_config_t* c) {
         case 24: case 32: break;
         default: return fail(MOE_ERR_UNSUPPORTED, "E=%d: E/32 must be one of 1-6,8,10,12,16,24,32", c->E);
     }
+    if (c->flags & ~(uint32_t)MOE_FLAG_TEST_STALL)
+        return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", c->flags);
     if (c->k < 1 || c->k > 32 || c->k > c->E)
         return fail(MOE_ERR_INVALID_ARG, "k=%d must be in [1, min(E, 32)]", c->k);
     if (c->I <= 0 || c->I % 128)
@@ -282,6 +284,7 @@ moe_status_t run_router_gemm(const moe_config_t* c, const void* x, const void* w
     p.split_stride = (long long)c->T * c->E;
     P.n_problems = 1;
     P.status = status;
+    P.test_stall = (c->flags & MOE_FLAG_TEST_STALL) ? 1 : 0;
     int sms = 0;
     MOE_TRY(sm_count(&sms));
     const int tiles = ((c->E + 127) / 128) * ((c->T + bn - 1) / bn) * split;

@@ -126,6 +126,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 const int kb0 = tl.kslice * nk;
                 for (int kb = kb0; kb < kb0 + nk; ++kb) {
                     if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    if (P.test_stall && blockIdx.x == 0 && issued == 0 && s == 0 && ph == 0) {
+                        // test of the bounded waits: this stage is never filled, so the
+                        // MMA's wait on it runs out; the stage is not marked issued
+                        if (++s == C::STAGES) { s = 0; ph ^= 1; }
+                        continue;
+                    }
                     uint8_t* st = smem + s * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
                     tma_load_2d(st, &p.tw, &full[s], kb * kBK, wrow);

@@ -117,6 +117,7 @@ struct GemmParams {
     GemmProblem p[2];
     int n_problems;
     int* status;
+    int test_stall;  // test only: CTA 0 never fills its first pipeline stage
 };
 
 // bn: token tile (16, 64 or 128).  grid: persistent CTAs.

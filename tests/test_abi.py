@@ -54,7 +54,7 @@ def test_workspace_size_and_offsets(B):
 @pytest.mark.parametrize("kw", [dict(H=100), dict(E=33), dict(E=0), dict(k=0), dict(k=300),
                                 dict(I=100), dict(n_group=3), dict(n_group=8, topk_group=9),
                                 dict(n_group=8, topk_group=1, k=33), dict(T=-1), dict(dtype=7),
-                                dict(n_shared=-1)])
+                                dict(n_shared=-1), dict(flags=0x80)])
 def test_invalid_configs_rejected(B, kw):
     with pytest.raises(B.MoeError):
         B.workspace_size(cfg(B, **kw))

@@ -213,3 +213,27 @@ def test_full_size_prefill_zipf(B, W):
 
 def test_full_size_grouped(B, W):
     full_size_check(B, W, "grouped", sample=4)
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives(B, W):
+    """Failure detection without a GPU fault: with MOE_FLAG_TEST_STALL the
+    router GEMM's first CTA never fills one pipeline stage, its bounded wait
+    runs out (~1 s), the kernel records a timeout and returns.  The host sees
+    MOE_ERR_TIMEOUT, and the next normal call on the same context is exact."""
+    wl = W.Workload("stall", T=64, H=1024, E=64, k=4, I=128, seed=6)
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl)
+    cfg.flags = B.MOE_FLAG_TEST_STALL
+    ws = B.alloc_workspace(cfg)
+    logits = torch.empty((wl.T, wl.E), device="cuda")
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), device="cuda")
+    B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], logits, idx, w, ws)
+    with pytest.raises(B.MoeError) as ei:
+        B.moe_check_device_status(ws)
+    assert ei.value.status == B.MOE_ERR_TIMEOUT
+    cfg.flags = 0
+    B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], logits, idx, w, ws)
+    B.moe_check_device_status(ws)
+    oidx, ow, _ = O.route(oracle_cfg(cfg), logits.cpu().numpy(), inp["bias"].cpu().numpy())
+    assert (idx.cpu().numpy() == oidx).all()
