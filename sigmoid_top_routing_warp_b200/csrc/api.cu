@@ -108,7 +108,7 @@ int router_split(const moe_config_t* c) {
 
 struct Layout {
     size_t status, logits, rpart, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash,
-        y, ysh, xq, sx, xpq, sxp, aq, sa, ashq, sash, total;
+        y, ysh, xq, sx, xpq, sxp, aq, sa, ashq, sash, toktiles, total;
 };
 
 Layout layout(const moe_config_t* c) {
@@ -132,6 +132,7 @@ Layout layout(const moe_config_t* c) {
     L.pos = take(n * 4);
     L.wperm = take(n * 4);
     L.tokstart = take((E + 1) * 4);
+    L.toktiles = take((n / 16 + E + 1) * 16);  // token tiles of at least 16 rows
     L.chunk = take((size_t)moe::permute_chunks((int)n) * E * 4);
     L.xperm = take(n * H * 2);
     L.a = take(n * I * 2);
@@ -468,6 +469,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
         MOE_TRY(make_pair_boxes(p.tx, g.x_perm, n, c->H, "gathered x"));
         p.seg = offsets;
         p.tok_start = g.tok_start;
+        p.tok_tiles = g.tok_tiles;
         p.n_exp = c->E;
         p.K = c->H;
         p.n_feat = c->I;
@@ -499,6 +501,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
         MOE_TRY(make_pair_boxes(p.tx, at<void>(ws, L.a), n, c->I, "expert activations"));
         p.seg = offsets;
         p.tok_start = g.tok_start;
+        p.tok_tiles = g.tok_tiles;
         p.n_exp = c->E;
         p.K = c->I;
         p.n_feat = c->H;
@@ -544,6 +547,7 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
     g.x_perm = at<uint16_t>(ws, L.xperm);
     g.w_perm = at<float>(ws, L.wperm);
     g.tok_start = at<int32_t>(ws, L.tokstart);
+    g.tok_tiles = at<int4>(ws, L.toktiles);
     g.T = c->T;
     g.k = c->k;
     g.H = c->H;

@@ -207,7 +207,13 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a, int gat
         }
         __syncthreads();
         const int total = block_exclusive_scan(v, a.E, tmp);
-        for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.tok_start[e] = v[e];
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+            a.tok_start[e] = v[e];
+            // token-tile table: one entry per bn-row tile of expert e
+            const int r0 = a.offsets[e], ne = a.offsets[e + 1] - r0;
+            for (int tt = 0; tt * a.bn < ne; ++tt)
+                a.tok_tiles[v[e] + tt] = make_int4(e, r0 + tt * a.bn, min(a.bn, ne - tt * a.bn), 0);
+        }
         if (threadIdx.x == 0) a.tok_start[a.E] = total;
         return;
     }

@@ -81,6 +81,17 @@ __device__ __forceinline__ bool ptile_at(const PairParams& P, int t, PTile& o) {
         }
         const int nf = (p.n_feat + feat_tile<EPI>() - 1) / feat_tile<EPI>();
         int e = 0, first = 0, ntok, seg0, seg1;
+        if (p.seg != nullptr && p.tok_tiles != nullptr) {
+            // feature tile innermost: t = token tile * nf + feature tile
+            const int j = t / nf;
+            const int4 info = __ldg(p.tok_tiles + j);
+            o.prob = pi;
+            o.exp = info.x;
+            o.f0 = (t - j * nf) * feat_tile<EPI>();
+            o.row0 = info.y;
+            o.nvalid = info.z;
+            return true;
+        }
         if (p.seg == nullptr) {
             ntok = (p.n_rows + kPairTokens - 1) / kPairTokens;
             seg0 = 0;
@@ -322,12 +333,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                 __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stage);  // [32 tokens][32]
                 float* stf = reinterpret_cast<float*>(stage);                 // [32 tokens][32]
                 float* outf = reinterpret_cast<float*>(p.out);
+                // routing weights of the tile's tokens, loaded once: lane l holds token c0 + l
+                float wpre[kPairTokens / 32];
+#pragma unroll
+                for (int i = 0; i < kPairTokens / 32; ++i) {
+                    const int c = 32 * i + lane;
+                    wpre[i] = (p.row_w && c < tl.nvalid) ? __ldg(p.row_w + tl.row0 + c) : 1.0f;
+                }
+#pragma unroll 1
                 for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld_32(tmem_base + ((uint32_t)(32 * q) << 16) + col0 + c0, r);
                     tmem_wait_ld();
-                    const int myrow = tl.row0 + c0 + lane;
-                    const float wv = (p.row_w && c0 + lane < tl.nvalid) ? __ldg(p.row_w + myrow) : 1.0f;
+                    float wv = wpre[0];
+#pragma unroll
+                    for (int i = 1; i < kPairTokens / 32; ++i)
+                        if (c0 == 32 * i) wv = wpre[i];
                     if (p.out_f32) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)

@@ -43,6 +43,7 @@ struct GatherArgs {
     uint16_t* x_perm;         // bf16 [T*k, H]
     float* w_perm;            // [T*k]
     int32_t* tok_start;       // [E + 1] token-tile prefix, tiles of bn rows
+    int4* tok_tiles;          // [T*k/bn + E] per token tile: {expert, first row, rows, 0}
     int T, k, H, E, bn;
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
@@ -141,6 +142,7 @@ struct PairProblem {
     CUtensorMap tx[kPairBoxes];
     const int32_t* seg;       // [n_exp + 1] token-row offsets, or null: rows [0, n_rows)
     const int32_t* tok_start; // [n_exp + 1] prefix of 256-token tiles, or null with seg
+    const int4* tok_tiles;    // with seg: token tile j = {expert, first row, rows, 0}
     int n_exp;
     int n_rows;
     int K;                    // multiple of 64
