@@ -64,15 +64,21 @@ def load_peaks():
 # ---------------------------------------------------------------- distributed
 
 def dist_setup():
+    """One process per GPU (RANK/LOCAL_RANK/WORLD_SIZE/MASTER_* from the
+    launcher).  NCCL when CUDA is present, gloo otherwise; a short timeout
+    so that ranks waiting for one another end with an error."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -85,12 +91,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, v: float) -> float:
+    """The job's time: the slowest rank's."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------- clocks
@@ -367,10 +381,21 @@ def oracle_sample(wl, inp, seconds: float):
     def u16(t):
         return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
+    fp8 = wl.dtype == "fp8"
+
+    def wcodes(t):  # expert weights as the oracle takes them: bf16 bits or e4m3 codes
+        return t.contiguous().cpu().numpy().astype(np.uint8) if fp8 else u16(t)
+
+    def wscale(name, sel=None):
+        if not fp8:
+            return None
+        t = inp[name] if sel is None else inp[name][sel]
+        return t.contiguous().cpu().float().numpy()
+
     threads = O.set_threads(os.cpu_count() or 1)
     wg = u16(inp["w_router"])
     bias = inp["bias"].cpu().numpy()
-    w13s, w2s = u16(inp["w13s"]), u16(inp["w2s"])
+    w13s, w2s = wcodes(inp["w13s"]), wcodes(inp["w2s"])
     n = max(1, min(wl.T, threads))
     spent, done, rounds = 0.0, 0, 0
     rng = np.random.default_rng(1)
@@ -380,7 +405,7 @@ def oracle_sample(wl, inp, seconds: float):
         oc = O.Config(T=len(toks), H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
                       n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
                       norm_topk_prob=wl.norm_topk_prob,
-                      routed_scaling_factor=wl.routed_scaling_factor)
+                      routed_scaling_factor=wl.routed_scaling_factor, fp8=fp8)
         # routing needs only W_g; the layer needs the experts these tokens use
         t0 = time.perf_counter()
         L = O.router_logits(oc, x, wg).astype(np.float32)
@@ -388,12 +413,14 @@ def oracle_sample(wl, inp, seconds: float):
         t_route = time.perf_counter() - t0
         used = np.unique(idx)
         sel = torch.as_tensor(used, device=inp["w13"].device)
-        w13, w2 = u16(inp["w13"][sel]), u16(inp["w2"][sel])
+        w13, w2 = wcodes(inp["w13"][sel]), wcodes(inp["w2"][sel])
         remap = np.full(wl.E, -1, np.int64)
         remap[used] = np.arange(used.size)
         oc2 = O.Config(**{**oc.__dict__, "E": int(used.size)})
         t1 = time.perf_counter()
-        O.layer(oc2, x, remap[idx].astype(np.int32), w, w13, w2, w13s, w2s)
+        O.layer(oc2, x, remap[idx].astype(np.int32), w, w13, w2, w13s, w2s,
+                w13_scale=wscale("w13_scale", sel), w2_scale=wscale("w2_scale", sel),
+                w13s_scale=wscale("w13s_scale"), w2s_scale=wscale("w2s_scale"))
         spent += t_route + time.perf_counter() - t1
         done += len(toks)
         rounds += 1
@@ -439,6 +466,7 @@ def main():
         line = run_reference(args, world, rank)
         if line is not None:
             print(json.dumps(line), flush=True)
+        dist_teardown(world)
         return
     peaks, peak_src = load_peaks()
     r = run_ours(args, world, rank, local)
@@ -508,9 +536,7 @@ def main():
                                 "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    dist_teardown(world)
 
 
 if __name__ == "__main__":
