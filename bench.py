@@ -194,8 +194,9 @@ class ClockSampler:
 # ---------------------------------------------------------------- ncu traffic
 
 KERNEL_SOURCES = {
-    "gate_up_decode": ["csrc/gemm.cu", "csrc/ptx.cuh", "csrc/kernels.cuh"],
+    "gate_up_decode": ["csrc/gemm.cu", "csrc/tiles.cuh", "csrc/ptx.cuh", "csrc/kernels.cuh"],
     "gate_up_prefill": ["csrc/gemm_pair.cu", "csrc/ptx.cuh", "csrc/kernels.cuh"],
+    "gate_up_fp8": ["csrc/gemm_fp8.cu", "csrc/tiles.cuh", "csrc/ptx.cuh", "csrc/kernels.cuh"],
 }
 
 
@@ -215,6 +216,7 @@ def profile_traffic(kind, algorithmic, workload):
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
+    ratio = None
     for name in sorted(os.listdir(pdir)):
         fields = {}
         with open(os.path.join(pdir, name)) as f:
@@ -227,11 +229,12 @@ def profile_traffic(kind, algorithmic, workload):
                     fields[k] = v.strip()
         if fields.get("kernel") != kind or fields.get("source_hash") != source_hash(kind):
             continue
+        # a capture of this exact workload wins over a ratio scaled from a smaller case
         if "traffic_bytes_per_launch" in fields and fields.get("workload") == workload:
             return float(fields["traffic_bytes_per_launch"])
-        if "traffic_over_algorithmic" in fields:
-            return float(fields["traffic_over_algorithmic"]) * algorithmic
-    return None
+        if "traffic_over_algorithmic" in fields and ratio is None:
+            ratio = float(fields["traffic_over_algorithmic"])
+    return None if ratio is None else ratio * algorithmic
 
 
 # ---------------------------------------------------------------- work model
@@ -476,7 +479,7 @@ def main():
     stage_names = r["B"].STAGE_NAMES
     g1_ms = float(r["stage_ms"][3])
     pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
-    kind = "gate_up_prefill" if pair else "gate_up_decode"
+    kind = "gate_up_fp8" if wl.dtype == "fp8" else "gate_up_prefill" if pair else "gate_up_decode"
     traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
     fp8 = wl.dtype == "fp8"
     if fp8:  # the fp8 tensor peak: the measured bf16 peaks x the nominal fp8/bf16 ratio 2
