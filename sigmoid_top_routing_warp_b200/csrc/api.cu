@@ -85,9 +85,15 @@ inline bool is_fp8(const moe_config_t* c) { return c->dtype == MOE_DTYPE_FP8_E4M
 
 // Token tile of the FP8 expert GEMMs (register accumulators: 16, 32 or 64
 // tokens; 64-token tiles use eight epilogue warps).
+// Token tile of the fp8 expert GEMMs: 16 / 32 / 64 rows for the weight-major
+// kernel, or the token-major kernel's 128 when experts average more than 48
+// rows and both contractions have K a multiple of 512.
 int fp8_bn(const moe_config_t* c) {
     const double avg = c->E ? (double)c->T * c->k / c->E : 0.0;
-    return avg <= 24.0 ? 16 : avg <= 48.0 ? 32 : 64;
+    if (avg <= 24.0) return 16;
+    if (avg <= 48.0) return 32;
+    if (c->H % 512 == 0 && c->I % 512 == 0) return moe::kFp8TokTile;
+    return 64;
 }
 
 int router_bn(const moe_config_t* c) { return c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128; }
@@ -254,6 +260,24 @@ moe_status_t make_map_u8(CUtensorMap* m, const void* ptr, size_t rows, size_t co
     return MOE_OK;
 }
 
+// fp32 block scales [rows][kbs] for the token-major fp8 kernel: box {4, box_rows}
+// (the scales of four K blocks of box_rows rows); kbs must be a multiple of 4.
+moe_status_t make_map_scales(CUtensorMap* m, const float* ptr, size_t rows, size_t kbs,
+                             int box_rows, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[2] = {kbs, rows};
+    cuuint64_t strides[1] = {kbs * 4};
+    cuuint32_t box[2] = {4, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
+
 // The token boxes of the CTA-pair kernels: 16, 32, 64 and 128 rows.
 moe_status_t make_pair_boxes(CUtensorMap* maps, const void* ptr, size_t rows, size_t cols,
                              const char* what) {
@@ -338,6 +362,27 @@ struct Weights {
 
 // FP8 layer: a0 quantisation of x, gather of codes and scales, then both
 // expert GEMMs on e4m3 operands with scale promotion (gemm_fp8.cu).
+// One fp8 expert GEMM launch: the weight-major kernel, or (bn = 128) the
+// token-major kernel with its scale tensor maps (problem 0 has `rows0`
+// activation rows, problem 1 `rows1`).
+moe_status_t launch_fp8(int epi, int bn, moe::GemmParams& P, int rows0, int rows1, int sms,
+                        cudaStream_t s, const char* what) {
+    if (bn == moe::kFp8TokTile) {
+        for (int pi = 0; pi < P.n_problems; ++pi) {
+            moe::GemmProblem& p = P.p[pi];
+            const size_t kbs = (size_t)p.K / 128;
+            MOE_TRY(make_map_scales(&p.tsx, p.x_scale, pi == 0 ? rows0 : rows1, kbs,
+                                    moe::kFp8TokTile, "activation scales"));
+            MOE_TRY(make_map_scales(&p.tsw, p.w_scale, (size_t)p.n_exp * p.w_rows / 128, kbs, 1,
+                                    "weight scales"));
+        }
+        MOE_CUDA(moe::launch_fp8_tm_gemm(epi, P, sms, s), what);
+        return MOE_OK;
+    }
+    MOE_CUDA(moe::launch_fp8_gemm(epi, bn, P, sms, s), what);
+    return MOE_OK;
+}
+
 moe_status_t run_expert_ffn_fp8(const moe_config_t* c, const void* x, const int32_t* offsets,
                                 const int32_t* pos, const float* topk_w, const Weights& W,
                                 void* y, void* y_shared, void* ws, cudaStream_t s,
@@ -410,7 +455,7 @@ moe_status_t run_expert_ffn_fp8(const moe_config_t* c, const void* x, const int3
         }
         P1.status = status;
     }
-    MOE_CUDA(moe::launch_fp8_gemm(moe::EPI_SWIGLU, bn, P1, sms, s), "fp8 gate/up GEMM launch");
+    MOE_TRY(launch_fp8(moe::EPI_SWIGLU, bn, P1, n, c->T, sms, s, "fp8 gate/up GEMM launch"));
     if (ev_gemm2) MOE_CUDA(cudaEventRecord(ev_gemm2, s), "event record");
 
     moe::GemmParams P2;
@@ -449,7 +494,7 @@ moe_status_t run_expert_ffn_fp8(const moe_config_t* c, const void* x, const int3
         }
         P2.status = status;
     }
-    MOE_CUDA(moe::launch_fp8_gemm(moe::EPI_SCALE, bn, P2, sms, s), "fp8 down GEMM launch");
+    MOE_TRY(launch_fp8(moe::EPI_SCALE, bn, P2, n, c->T, sms, s, "fp8 down GEMM launch"));
     return MOE_OK;
 }
 

@@ -1,0 +1,360 @@
+// gemm_fp8_tm.cu -- token-major grouped expert GEMMs on e4m3 operands with
+// fp32 block scales, for batches with many tokens per expert (steps a6-a8 of
+// the FP8 layer), tcgen05 kind::f8f6f4 + TMEM.
+//
+// Source of the operation: "Xiaohongshu dots3 note Open Source Deep Dive",
+// §8.2 (gmm1 -> swiglu -> gmm2) and §3.2 (FP8 weights); "dots3-note 架构深度解析"
+// (mlqm.cn), 部署实战 (FP8 weights).  Recipe: weights e4m3 with one fp32 scale
+// per 128x128 block; activations e4m3 with one fp32 scale per row and 128
+// columns (quant.cu).
+//
+// The scales are arbitrary fp32 values, so every 128-wide K block is one MMA
+// group into a tensor-memory partial that the epilogue promotes into fp32
+// register accumulators:  acc[r, f] += s_x(r, kb) * s_w(f / 128, kb) * P_kb[r, f].
+// Here the tokens are the MMA's M operand (128 rows, one per TMEM lane) and
+// the weights its N operand (256 rows: 128 gate + 128 up features, or 256
+// output features).  Each epilogue thread then owns one token row, so the
+// scale of a K block is one product per thread and promotion is one FMA per
+// element, with no cross-lane traffic.  (gemm_fp8.cu puts the weights in M,
+// which suits a few tokens per expert but makes the scale vary along the
+// accumulator's columns.)
+//
+// Roles (18 warps): warp 0 issues TMA loads (operands per K block; the
+// scales of four K blocks at a time into a small ring: s_x for the tile's
+// 128 rows as one {4, 128} box, s_w as two {4, 1} boxes), warp 1 allocates
+// tensor memory and issues the MMAs (one thread), warps 2-17 promote and
+// finish: warp w reads TMEM lane quadrant w % 4 and column group (w - 2) / 4.
+// Two 256-column partial buffers let the MMAs of block kb+1 run while block
+// kb is promoted.
+//
+// EPI_SWIGLU: a = SiLU(gate) * up, quantised per token over the tile's 128
+// features (one e4m3 block of A); the four column groups exchange their
+// maxima through shared memory under a bounded mbarrier.
+// EPI_SCALE: y = acc * routing weight, bf16 (or fp32 for the shared expert).
+//
+// Waits are bounded as in gemm.cu (DEV_STATUS_TIMEOUT, abort flag, drain).
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tiles.cuh"
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+namespace moe {
+
+namespace {
+
+constexpr int kTMTok = 128;                    // token rows per tile (MMA M)
+constexpr int kTMN = 256;                      // weight rows per tile (MMA N)
+constexpr int kTMBK = 128;                     // K per stage: one scale block, 128 B rows
+constexpr int kTMABytes = kTMTok * kTMBK;      // 16 KB of token codes
+constexpr int kTMBBytes = kTMN * kTMBK;        // 32 KB of weight codes
+constexpr int kTMStage = kTMABytes + kTMBBytes;
+constexpr int kTMStages = 4;
+constexpr int kTMGroup = 4;                    // K blocks per scale fetch
+constexpr int kTMSSlots = 3;                   // scale ring depth
+constexpr int kTMSSlot = 2304;                 // s_x [128][4] at 0, s_w rows at 2048 and 2176
+constexpr int kTMEpiWarps = 16;
+constexpr int kTMThreads = 64 + 32 * kTMEpiWarps;
+constexpr int kTMNP = 2;                       // partial buffers of kTMN columns
+constexpr int kTMAmaxBytes = 2 * 4 * kTMTok * 4;  // [2 parities][4 column groups][128 rows]
+constexpr int kTMBarBytes = 256;
+constexpr int kTMSmem = 1024 + kTMStages * kTMStage + kTMSSlots * kTMSSlot + kTMAmaxBytes +
+                        kTMBarBytes;
+// kind::f8f6f4: fp32 accumulator, e4m3 A and B (format 0), K-major, M = 128, N = 256
+constexpr uint32_t kTMIdesc = (1u << 4) | ((uint32_t)(kTMN >> 3) << 17) | ((uint32_t)(kTMTok >> 4) << 24);
+static_assert(kTMSmem <= 232448, "shared memory budget");
+static_assert(kTMStage % 1024 == 0 && kTMSSlot % 128 == 0, "TMA destinations stay aligned");
+
+__device__ __forceinline__ void tm_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(kTMIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// Promote 16 columns of a partial: acc[j] += s * P[j].
+__device__ __forceinline__ void tm_promote16(uint32_t taddr, float s, float* acc) {
+    uint32_t r[16];
+    tmem_ld_16(taddr, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = fmaf(s, __uint_as_float(r[j]), acc[j]);
+}
+
+}  // namespace
+
+template <int EPI>
+__global__ void __launch_bounds__(kTMThreads, 1)
+    fp8_tm_gemm_kernel(const __grid_constant__ GemmParams P) {
+    constexpr int FSZ = EPI == EPI_SWIGLU ? 128 : 256;  // output features per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sring = smem + kTMStages * kTMStage;
+    float* amax_sm = reinterpret_cast<float*>(sring + kTMSSlots * kTMSSlot);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(amax_sm) + kTMAmaxBytes);
+    uint64_t* empty = full + kTMStages;
+    uint64_t* sfull = empty + kTMStages;     // scale slot loaded (TMA)
+    uint64_t* sempty = sfull + kTMSSlots;    // scale slot read (16 epilogue warps)
+    uint64_t* pfull = sempty + kTMSSlots;    // partial ready (MMA -> epilogue)
+    uint64_t* pempty = pfull + kTMNP;        // partial read (16 epilogue warps)
+    uint64_t* amax_bar = pempty + kTMNP;     // [2] row maxima of all column groups written
+    uint64_t* mma_done = amax_bar + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTMStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kTMSSlots; ++s) {
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sempty[s], kTMEpiWarps);
+        }
+        for (int b = 0; b < kTMNP; ++b) {
+            mbar_init(&pfull[b], 1);
+            mbar_init(&pempty[b], kTMEpiWarps);
+        }
+        for (int b = 0; b < 2; ++b) mbar_init(&amax_bar[b], kTMEpiWarps);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        for (int pi = 0; pi < P.n_problems; ++pi) {
+            tma_prefetch_desc(&P.p[pi].tw);
+            tma_prefetch_desc(&P.p[pi].tx);
+            tma_prefetch_desc(&P.p[pi].tsx);
+            tma_prefetch_desc(&P.p[pi].tsw);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTMNP * kTMN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int ntiles = total_tiles(P, kTMTok, FSZ);
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int s = 0, ss = 0;
+            uint32_t ph = 0, sph = 0, issued = 0, sissued = 0, last_ph = 0, slast_ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                Tile tl;
+                tile_at(P, kTMTok, t, tl, FSZ);
+                const GemmProblem& p = P.p[tl.prob];
+                const int nk = p.K / kTMBK;
+                // weight rows of the tile's two 128-row halves and their scale-block rows
+                const int w0 = tl.exp * p.w_rows + tl.f0;
+                const int w1 = EPI == EPI_SWIGLU ? w0 + p.n_feat : w0 + 128;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (kb % kTMGroup == 0) {
+                        if (!wait_bar(&sempty[ss], sph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                        uint8_t* sl = sring + ss * kTMSSlot;
+                        mbar_arrive_expect_tx(&sfull[ss], kTMTok * 16 + 2 * 16);
+                        tma_load_2d(sl, &p.tsx, &sfull[ss], kb, tl.row0);
+                        tma_load_2d(sl + 2048, &p.tsw, &sfull[ss], kb, w0 / 128);
+                        tma_load_2d(sl + 2176, &p.tsw, &sfull[ss], kb, w1 / 128);
+                        sissued |= 1u << ss;
+                        slast_ph = (slast_ph & ~(1u << ss)) | (sph << ss);
+                        if (++ss == kTMSSlots) { ss = 0; sph ^= 1; }
+                    }
+                    if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    uint8_t* st = smem + s * kTMStage;
+                    mbar_arrive_expect_tx(&full[s], kTMStage);
+                    tma_load_2d(st, &p.tx, &full[s], kb * kTMBK, tl.row0);
+                    tma_load_2d(st + kTMABytes, &p.tw, &full[s], kb * kTMBK, w0);
+                    tma_load_2d(st + kTMABytes + kTMBBytes / 2, &p.tw, &full[s], kb * kTMBK, w1);
+                    issued |= 1u << s;
+                    last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                    if (++s == kTMStages) { s = 0; ph ^= 1; }
+                }
+            }
+            // drain: every issued copy lands before the CTA exits
+            for (int i = 0; i < kTMStages; ++i)
+                if (issued >> i & 1u) wait_bar(&full[i], last_ph >> i & 1u, abort_flag, P.status, true);
+            for (int i = 0; i < kTMSSlots; ++i)
+                if (sissued >> i & 1u) wait_bar(&sfull[i], slast_ph >> i & 1u, abort_flag, P.status, true);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer: one group per K block
+        if (lane == 0) {
+            int s = 0, pb = 0;
+            uint32_t ph = 0, pph = 0;
+            bool ok = true, any = false;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                Tile tl;
+                tile_at(P, kTMTok, t, tl, FSZ);
+                const int nk = P.p[tl.prob].K / kTMBK;
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (!wait_bar(&pempty[pb], pph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    if (!wait_bar(&full[s], ph, abort_flag, P.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(smem + s * kTMStage);
+                    const uint32_t d = tmem_base + pb * kTMN;
+#pragma unroll
+                    for (int kk = 0; kk < kTMBK / 32; ++kk)
+                        tm_mma_f8(d, smem_desc_k_sw128(st + kk * 32),
+                                  smem_desc_k_sw128(st + kTMABytes + kk * 32), kk != 0);
+                    tc_commit(&empty[s]);
+                    tc_commit(&pfull[pb]);
+                    any = true;
+                    if (++s == kTMStages) { s = 0; ph ^= 1; }
+                    if (++pb == kTMNP) { pb = 0; pph ^= 1; }
+                }
+            }
+            if (any) {
+                tc_commit(mma_done);
+                wait_bar(mma_done, 0, abort_flag, P.status, true);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue: promote, then finish the tile
+        const int q = warp & 3;              // TMEM lane quadrant: rows 32q .. 32q + 31
+        const int g = (warp - 2) >> 2;       // column group
+        const int tok = 32 * q + lane;       // this thread's row of the tile
+        // accumulator columns: SWIGLU gate [32g, 32g+32) and up [128+32g, ...);
+        // SCALE [64g, 64g+64), both halves in weight-scale block g / 2
+        const uint32_t ca = EPI == EPI_SWIGLU ? 32 * g : 64 * g;
+        const uint32_t cb = EPI == EPI_SWIGLU ? 128 + 32 * g : 64 * g + 32;
+        const int swa = EPI == EPI_SWIGLU ? 0 : (g >> 1);
+        const int swb = EPI == EPI_SWIGLU ? 1 : (g >> 1);
+        int pb = 0, ss = 0, tile_no = 0;
+        uint32_t pph = 0, sph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tile_no) {
+            Tile tl;
+            tile_at(P, kTMTok, t, tl, FSZ);
+            const GemmProblem& p = P.p[tl.prob];
+            const int nk = p.K / kTMBK;
+            const bool valid = tok < tl.nvalid;
+            const int row = tl.row0 + tok;
+            float acc[64];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+            for (int kb0 = 0; kb0 < nk && ok; kb0 += kTMGroup) {
+                if (!wait_bar(&sfull[ss], sph, abort_flag, P.status)) { ok = false; break; }
+                const uint8_t* sl = sring + ss * kTMSSlot;
+                const float4 sx = reinterpret_cast<const float4*>(sl)[tok];
+                const float4 wa = *reinterpret_cast<const float4*>(sl + 2048 + 128 * swa);
+                const float4 wb = *reinterpret_cast<const float4*>(sl + 2048 + 128 * swb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sempty[ss]);
+                if (++ss == kTMSSlots) { ss = 0; sph ^= 1; }
+                const float sxs[4] = {sx.x, sx.y, sx.z, sx.w};
+                const float was[4] = {wa.x, wa.y, wa.z, wa.w};
+                const float wbs[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                for (int i = 0; i < kTMGroup; ++i) {
+                    if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + pb * kTMN;
+                    const float sa = sxs[i] * was[i], sb = sxs[i] * wbs[i];
+                    tm_promote16(tb + ca, sa, acc);
+                    tm_promote16(tb + ca + 16, sa, acc + 16);
+                    tm_promote16(tb + cb, sb, acc + 32);
+                    tm_promote16(tb + cb + 16, sb, acc + 48);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pempty[pb]);
+                    if (++pb == kTMNP) { pb = 0; pph ^= 1; }
+                }
+            }
+            if (!ok) break;
+            if (EPI == EPI_SWIGLU) {
+                // a = SiLU(gate) * up for features f0 + 32g .. + 31 of this row
+                float m = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    acc[j] = silu(acc[j]) * acc[32 + j];
+                    m = fmaxf(m, fabsf(acc[j]));
+                }
+                const int par = tile_no & 1;
+                amax_sm[(par * 4 + g) * kTMTok + tok] = m;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&amax_bar[par]);
+                if (!wait_bar(&amax_bar[par], (tile_no >> 1) & 1, abort_flag, P.status)) break;
+                const float* all = amax_sm + par * 4 * kTMTok + tok;
+                const float amax = fmaxf(fmaxf(all[0], all[kTMTok]), fmaxf(all[2 * kTMTok], all[3 * kTMTok]));
+                const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                if (valid) {
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        uint32_t v = 0;
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            v |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(acc[4 * w + b], sc),
+                                                                  __NV_SATFINITE, __NV_E4M3) << (8 * b);
+                        packed[w] = v;
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(p.out_q + (size_t)row * p.ld_out + tl.f0 + 32 * g);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    if (g == 0) p.out_scale[(size_t)row * (p.ld_out / 128) + tl.f0 / 128] = sc;
+                }
+            } else {
+                const int f = tl.f0 + 64 * g;
+                if (valid && f < p.n_feat) {
+                    const float wr = p.row_w ? __ldg(p.row_w + row) : 1.0f;
+                    if (p.out_f32) {
+                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                                                (size_t)row * p.ld_out + f);
+#pragma unroll
+                        for (int v = 0; v < 16; ++v)
+                            dst[v] = make_float4(acc[4 * v] * wr, acc[4 * v + 1] * wr,
+                                                 acc[4 * v + 2] * wr, acc[4 * v + 3] * wr);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                              (size_t)row * p.ld_out + f);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[8 * v + 2 * h] * wr,
+                                                                                acc[8 * v + 2 * h + 1] * wr);
+                                w4[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
+                            dst[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTMNP * kTMN);
+}
+
+template <int EPI>
+static cudaError_t launch_tm(const GemmParams& params, int grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(fp8_tm_gemm_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kTMSmem);
+    if (e != cudaSuccess) return e;
+    fp8_tm_gemm_kernel<EPI><<<grid, kTMThreads, kTMSmem, s>>>(params);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cudaStream_t s) {
+    if (epi == EPI_SWIGLU) return launch_tm<EPI_SWIGLU>(params, grid, s);
+    if (epi == EPI_SCALE) return launch_tm<EPI_SCALE>(params, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -112,6 +112,10 @@ struct GemmProblem {
     const float* x_scale;     // [rows][K/128] activation scales
     uint8_t* out_q;           // EPI_SWIGLU: e4m3 codes [rows, ld_out]
     float* out_scale;         // EPI_SWIGLU: scales [rows, ld_out/128]
+    // token-major fp8 kernel: the same scales as fp32 2-D tensor maps,
+    // x_scale box {4, 128} and w_scale box {4, 1}
+    CUtensorMap tsx;
+    CUtensorMap tsw;
 };
 
 struct GemmParams {
@@ -162,7 +166,13 @@ struct PairParams {
 cudaError_t launch_pair_gemm(int epi, const PairParams& params, int grid, cudaStream_t s);
 
 // FP8 grouped GEMM (single CTA, weights as the M operand): EPI_SWIGLU
-// (writes e4m3 codes + scales of A) or EPI_SCALE (bf16 / fp32 out).  bn 16 or 32.
+// (writes e4m3 codes + scales of A) or EPI_SCALE (bf16 / fp32 out).  bn 16, 32, 64.
 cudaError_t launch_fp8_gemm(int epi, int bn, const GemmParams& params, int grid, cudaStream_t s);
+
+// Token-major FP8 grouped GEMM (tokens as the M operand, 128-row token tiles;
+// features per tile: 128 for EPI_SWIGLU, 256 for EPI_SCALE).  Needs K a
+// multiple of 512, n_feat a multiple of 128, and the tsx / tsw maps.
+constexpr int kFp8TokTile = 128;
+cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cudaStream_t s);
 
 }  // namespace moe

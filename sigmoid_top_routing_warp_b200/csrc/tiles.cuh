@@ -12,8 +12,9 @@ struct Tile {
     int prob, exp, row0, nvalid, f0, kslice;
 };
 
-__device__ __forceinline__ int problem_tiles(const GemmProblem& p, int bn) {
-    const int nf = (p.n_feat + 127) / 128;
+// fsz: output features per tile (128, or 256 for the token-major fp8 kernel).
+__device__ __forceinline__ int problem_tiles(const GemmProblem& p, int bn, int fsz = 128) {
+    const int nf = (p.n_feat + fsz - 1) / fsz;
     if (p.seg == nullptr) return nf * ((p.n_rows + bn - 1) / bn) * max(p.k_split, 1);
     return nf * __ldg(p.tok_start + p.n_exp);
 }
@@ -21,15 +22,16 @@ __device__ __forceinline__ int problem_tiles(const GemmProblem& p, int bn) {
 // Tile t of the launch -> (problem, expert, token rows, feature tile).
 // Order inside a problem: expert, then feature tile, then token tile, so that
 // CTAs working at the same time share weight tiles through L2.
-__device__ __forceinline__ bool tile_at(const GemmParams& P, int bn, int t, Tile& o) {
+__device__ __forceinline__ bool tile_at(const GemmParams& P, int bn, int t, Tile& o,
+                                        int fsz = 128) {
     for (int pi = 0; pi < P.n_problems; ++pi) {
         const GemmProblem& p = P.p[pi];
-        const int n = problem_tiles(p, bn);
+        const int n = problem_tiles(p, bn, fsz);
         if (t >= n) {
             t -= n;
             continue;
         }
-        const int nf = (p.n_feat + 127) / 128;
+        const int nf = (p.n_feat + fsz - 1) / fsz;
         int e = 0, first = 0, ntok, seg0, seg1;
         o.kslice = 0;
         if (p.seg == nullptr && p.k_split > 1) {
@@ -57,7 +59,7 @@ __device__ __forceinline__ bool tile_at(const GemmParams& P, int bn, int t, Tile
         const int ft = local / ntok, tt = local - ft * ntok;
         o.prob = pi;
         o.exp = e;
-        o.f0 = ft * 128;
+        o.f0 = ft * fsz;
         o.row0 = seg0 + tt * bn;
         o.nvalid = min(bn, seg1 - o.row0);
         return true;
@@ -65,9 +67,9 @@ __device__ __forceinline__ bool tile_at(const GemmParams& P, int bn, int t, Tile
     return false;
 }
 
-__device__ __forceinline__ int total_tiles(const GemmParams& P, int bn) {
+__device__ __forceinline__ int total_tiles(const GemmParams& P, int bn, int fsz = 128) {
     int n = 0;
-    for (int pi = 0; pi < P.n_problems; ++pi) n += problem_tiles(P.p[pi], bn);
+    for (int pi = 0; pi < P.n_problems; ++pi) n += problem_tiles(P.p[pi], bn, fsz);
     return n;
 }
 
