@@ -445,6 +445,62 @@ void orc_layer(const orc_config* cfg, const uint16_t* x, const int32_t* idx, con
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Pre-norm around the layer (next to the layer, not inside it):            */
+/*   [DEEP] §3.3 layer diagram: "Residual + RMSNorm" feeds the MoE FFN and   */
+/*   "Residual + Output" follows it;                                         */
+/*   [DOTS1] config table: rms_norm_eps = 1e-6; source-notes paragraph: the  */
+/*   variance is taken in fp32, the row is scaled by its reciprocal square   */
+/*   root, then multiplied by the weight.                                    */
+/* Reading: u[t,h] = gamma[h] * h[t,h] / sqrt(mean_h h[t,h]^2 + eps), here   */
+/* in fp64 from the bf16 operands and rounded once to bf16 (RNE).            */
+/* ------------------------------------------------------------------------ */
+
+/* binary64 -> bf16, round to nearest even, in one step (no detour through
+ * binary32, which would round twice).  bf16 keeps 8 significant bits;
+ * below 2^-126 its grid is the subnormal spacing 2^-133. */
+uint16_t orc_f64_to_bf16(double d) {
+    if (isnan(d)) return 0x7FC0u;
+    const uint16_t sign = signbit(d) ? 0x8000u : 0u;
+    const double a = fabs(d);
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e); /* a = m * 2^e, m in [0.5, 1): leading bit has weight 2^(e-1) */
+    double q;
+    if (e - 1 < -126)
+        q = ldexp(rint(ldexp(a, 133)), -133);
+    else
+        q = ldexp(rint(ldexp(a, 8 - e)), e - 8);
+    if (q >= ldexp(1.0, 128)) return sign | 0x7F80u; /* overflow to infinity */
+    float f = (float)q; /* exact: q has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)(u >> 16);
+}
+
+/* h, u: bf16 [T,H]; gamma: bf16 [H]; r (optional): per row 1/sqrt(ms + eps). */
+void orc_rmsnorm(int T, int H, const uint16_t* h, const uint16_t* gamma, double eps, uint16_t* u,
+                 double* r) {
+    for (int t = 0; t < T; ++t) {
+        const uint16_t* row = h + (size_t)t * H;
+        double ss = 0.0;
+        for (int i = 0; i < H; ++i) {
+            const double v = (double)orc_bf16_to_f32(row[i]);
+            ss += v * v;
+        }
+        const double rt = 1.0 / sqrt(ss / H + eps);
+        if (r) r[t] = rt;
+        for (int i = 0; i < H; ++i)
+            u[(size_t)t * H + i] = orc_f64_to_bf16((double)orc_bf16_to_f32(gamma[i]) *
+                                                   ((double)orc_bf16_to_f32(row[i]) * rt));
+    }
+}
+
+/* Element-wise binary64 -> bf16 (for the rounding pins). */
+void orc_f64_to_bf16_n(const double* x, uint16_t* y, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) y[i] = orc_f64_to_bf16(x[i]);
+}
+
 /* Thread count for the OpenMP loops above (returns the count in effect). */
 int orc_set_threads(int n) {
 #ifdef _OPENMP

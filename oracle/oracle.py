@@ -94,6 +94,12 @@ def lib():
         _lib.orc_quant_act_e4m3.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
         _lib.orc_layer.restype = None
         _lib.orc_layer.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 12 + [ctypes.c_int, P]
+        _lib.orc_f64_to_bf16.restype = ctypes.c_uint16
+        _lib.orc_f64_to_bf16.argtypes = [ctypes.c_double]
+        _lib.orc_f64_to_bf16_n.restype = None
+        _lib.orc_f64_to_bf16_n.argtypes = [P, P, ctypes.c_int64]
+        _lib.orc_rmsnorm.restype = None
+        _lib.orc_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, P, P, ctypes.c_double, P, P]
         _lib.orc_set_threads.restype = ctypes.c_int
         _lib.orc_set_threads.argtypes = [ctypes.c_int]
     return _lib
@@ -229,3 +235,40 @@ def layer(cfg: Config, x_bf16, idx, w, w13, w2, w13s, w2s, tokens=None,
                     _p(sc[1]), _p(w13s), _p(sc[2]), _p(w2s), _p(sc[3]), _p(tokens),
                     int(tokens.size), _p(out))
     return out
+
+
+def f64_to_bf16(d) -> np.ndarray:
+    """binary64 -> bf16 bits, round to nearest even in one step."""
+    d = _c(d, np.float64)
+    y = np.empty(d.shape, dtype=np.uint16)
+    lib().orc_f64_to_bf16_n(_p(d), _p(y), d.size)
+    return y
+
+
+def rmsnorm(h_bf16, gamma_bf16, eps: float) -> tuple[np.ndarray, np.ndarray]:
+    """Pre-norm of the layer input: (u bf16 bits [T, H], r = 1/sqrt(ms + eps) [T]).
+
+    u = bf16(gamma * h / sqrt(mean(h^2) + eps)), evaluated in fp64, one rounding.
+    """
+    h = _c(h_bf16, np.uint16)
+    g = _c(gamma_bf16, np.uint16)
+    T, H = h.shape
+    assert g.size == H
+    u = np.empty((T, H), dtype=np.uint16)
+    r = np.empty(T, dtype=np.float64)
+    lib().orc_rmsnorm(T, H, _p(h), _p(g), float(eps), _p(u), _p(r))
+    return u, r
+
+
+def block(cfg: Config, h_bf16, gamma_bf16, eps: float, idx, w, w13, w2, w13s, w2s,
+          tokens=None, **scales) -> np.ndarray:
+    """fp64 output of one pre-norm block, h + layer(RMSNorm(h)), for the given
+    routing (rows `tokens`)."""
+    h = _c(h_bf16, np.uint16)
+    u, _ = rmsnorm(h, gamma_bf16, eps)
+    if tokens is None:
+        tokens = np.arange(cfg.T, dtype=np.int32)
+    tokens = _c(tokens, np.int32)
+    moe = layer(cfg, u, idx, w, w13, w2, w13s, w2s, tokens=tokens, **scales)
+    hv = (h[tokens].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return hv + moe

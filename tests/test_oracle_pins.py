@@ -452,3 +452,101 @@ def test_layer_fp8_against_dense_dequantised_brute_force():
     # A is quantised from its fp32 rounding in the oracle and from fp64 here:
     # a code can move by one step at a rounding boundary, hence the tolerance
     assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-3
+
+
+# ---------------------------------------------------------------- pre-norm block
+def _bf16_value(b):
+    return float(np.array([int(b) << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def _nearest_bf16_exact(d: float) -> int:
+    """Brute force: the bf16 pattern nearest to d in exact rational arithmetic,
+    ties to the even pattern (independent of the oracle's scaling method)."""
+    x = Fraction(d)
+    f = np.array([d], dtype=np.float32).view(np.uint32)[0] >> 16  # a nearby pattern
+    best = None
+    for c in range(int(f) - 2, int(f) + 3):
+        c &= 0xFFFF
+        v = _bf16_value(c)
+        if not math.isfinite(v):
+            continue
+        err = abs(Fraction(v) - x)
+        key = (err, c & 1)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return best[1]
+
+
+def test_f64_to_bf16_is_nearest_even():
+    rng = np.random.default_rng(7)
+    vals = list(rng.standard_normal(300) * 10.0 ** rng.integers(-30, 30, 300))
+    vals += [1.0 + 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -40, 1.0 + 3 * 2.0 ** -8,
+             -(1.0 + 2.0 ** -8), 2.0 ** -130, 3 * 2.0 ** -134, 2.0 ** -127 * 1.5]
+    got = O.f64_to_bf16(np.array(vals))
+    for d, g in zip(vals, got):
+        assert int(g) == _nearest_bf16_exact(d), (d, hex(int(g)))
+    assert int(O.f64_to_bf16(np.array([1e39]))[0]) == 0x7F80
+    assert int(O.f64_to_bf16(np.array([-0.0]))[0]) == 0x8000
+
+
+def test_rmsnorm_closed_forms():
+    H = 64
+    one = np.full(H, 0x3F80, dtype=np.uint16)
+    two = np.full(H, 0x4000, dtype=np.uint16)
+    # constant row c: u = gamma * c / sqrt(c^2 + eps)
+    c = O.f32_to_bf16(np.array([3.0], dtype=np.float32))[0]
+    h = np.full((1, H), c, dtype=np.uint16)
+    u, r = O.rmsnorm(h, two, 1e-6)
+    exp_u = _nearest_bf16_exact(2.0 * 3.0 / math.sqrt(9.0 + 1e-6))
+    assert (u == exp_u).all() and abs(r[0] - 1.0 / math.sqrt(9.0 + 1e-6)) < 1e-15
+    # one non-zero entry v in a row of H: mean square v^2 / H, so u = sqrt(H) sign(v)
+    h = np.zeros((1, H), dtype=np.uint16)
+    h[0, 5] = O.f32_to_bf16(np.array([-0.75], dtype=np.float32))[0]
+    u, _ = O.rmsnorm(h, one, 0.0)
+    assert _bf16_value(u[0, 5]) == -8.0 and (np.delete(u[0], 5) == 0).all()
+    # eps-dominated rows: |h| << sqrt(eps) gives u ~ h / sqrt(eps)
+    h = np.full((1, H), O.f32_to_bf16(np.array([1e-6], dtype=np.float32))[0], dtype=np.uint16)
+    hv = _bf16_value(h[0, 0])
+    u, _ = O.rmsnorm(h, one, 1e-6)
+    assert int(u[0, 0]) == _nearest_bf16_exact(hv / math.sqrt(hv * hv + 1e-6))
+
+
+def test_rmsnorm_invariants():
+    rng = np.random.default_rng(3)
+    T, H = 6, 256
+    h = O.f32_to_bf16(rng.standard_normal((T, H)).astype(np.float32))
+    g1 = np.full(H, 0x3F80, dtype=np.uint16)
+    u, _ = O.rmsnorm(h, g1, 0.0)
+    uv = (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # unit mean square up to bf16 rounding
+    assert np.abs((uv ** 2).mean(axis=1) - 1.0).max() < 4e-3
+    # exact invariance under a power-of-two rescale of the row (eps = 0)
+    h2 = O.f32_to_bf16(((h.astype(np.uint32) << 16).view(np.float32) * 8.0).astype(np.float32))
+    u2, _ = O.rmsnorm(h2, g1, 0.0)
+    assert (u2 == u).all()
+    # gamma scales the output column-wise (a power of two: exact)
+    g4 = np.full(H, 0x4080, dtype=np.uint16)  # 4.0
+    u4, _ = O.rmsnorm(h, g4, 0.0)
+    assert np.array_equal((u4.astype(np.uint32) << 16).view(np.float32),
+                          4.0 * (u.astype(np.uint32) << 16).view(np.float32))
+
+
+def test_block_is_residual_plus_layer():
+    rng = np.random.default_rng(11)
+    cfg = O.Config(T=5, H=128, E=32, k=2, I=64, n_shared=1)
+    h = O.f32_to_bf16(rng.standard_normal((cfg.T, cfg.H)).astype(np.float32))
+    gamma = O.f32_to_bf16((1.0 + 0.1 * rng.standard_normal(cfg.H)).astype(np.float32))
+    w13 = O.f32_to_bf16((0.05 * rng.standard_normal((cfg.E, 2 * cfg.I, cfg.H))).astype(np.float32))
+    w2 = O.f32_to_bf16((0.05 * rng.standard_normal((cfg.E, cfg.H, cfg.I))).astype(np.float32))
+    w13s = O.f32_to_bf16((0.05 * rng.standard_normal((2 * cfg.I, cfg.H))).astype(np.float32))
+    w2s = O.f32_to_bf16((0.05 * rng.standard_normal((cfg.H, cfg.I))).astype(np.float32))
+    idx = np.stack([rng.choice(cfg.E, cfg.k, replace=False) for _ in range(cfg.T)]).astype(np.int32)
+    w = np.full((cfg.T, cfg.k), 0.5, dtype=np.float32)
+    out = O.block(cfg, h, gamma, 1e-6, idx, w, w13, w2, w13s, w2s)
+    u, _ = O.rmsnorm(h, gamma, 1e-6)
+    hv = (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(out, hv + O.layer(cfg, u, idx, w, w13, w2, w13s, w2s))
+    # zero expert weights: the block returns its input exactly
+    z13, z2 = np.zeros_like(w13), np.zeros_like(w2)
+    out0 = O.block(cfg, h, gamma, 1e-6, idx, w, z13, z2, np.zeros_like(w13s), np.zeros_like(w2s))
+    np.testing.assert_array_equal(out0, hv)
