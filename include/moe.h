@@ -234,11 +234,43 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
                          void* out, void* ws, size_t ws_bytes, void* const* stage_events,
                          moe_stream_t stream);
 
+/* Pre-norm of the block input.  Pages: Deep Dive §3.3 layer diagram (the
+ * "Residual + RMSNorm" box ahead of the MoE FFN); Dots1 config table
+ * (rms_norm_eps = 1e-6) and its source notes (variance in fp32, scaling by
+ * the reciprocal square root, then the weight).  Per row t, in fp32 with
+ * correctly rounded divide and square root:
+ *   u[t, :] = bf16( gamma * (h[t, :] * r_t) ),
+ *   r_t = 1 / sqrt(sum_i h[t, i]^2 / H + eps)
+ *   h     bf16 [T, H]  (16-byte aligned)
+ *   gamma bf16 [H]     norm weight
+ *   u     bf16 [T, H]  output; must not overlap h
+ *   eps   finite, >= 0 (the pages' value is 1e-6)
+ * Only cfg->T and cfg->H are read; H must be a multiple of 8. */
+moe_status_t moe_rmsnorm(const moe_config_t* cfg, const void* h, const void* gamma, float eps,
+                         void* u, moe_stream_t stream);
+
+/* One pre-norm MoE block, out = h + MoE(RMSNorm(h)): the same diagram's
+ * "Residual + RMSNorm" -> MoE FFN -> "Residual + Output".  h is the residual
+ * stream (bf16 [T, H]); the layer runs on u = RMSNorm(h) (as moe_rmsnorm,
+ * kept in the workspace, see moe_workspace_offset item 8), and the combine
+ * adds h in the same fp32 sum as the expert outputs, before the single bf16
+ * rounding:  out[t] = bf16( sum_j y[pos[t*k+j]] + y_shared[t] + h[t] ).
+ * out may be h itself (in-place residual update); otherwise it must not
+ * overlap h.  Other arguments as moe_forward; stage 0 of stage_events also
+ * covers the norm. */
+moe_status_t moe_forward_block(const moe_config_t* cfg, const void* h, const void* gamma,
+                               float eps, const void* w_router, const float* bias,
+                               const void* w13, const float* w13_scale, const void* w2,
+                               const float* w2_scale, const void* w13s, const float* w13s_scale,
+                               const void* w2s, const float* w2s_scale, void* out, void* ws,
+                               size_t ws_bytes, void* const* stage_events, moe_stream_t stream);
+
 /* Device byte offsets, inside the workspace, of the intermediates that
  * moe_forward leaves there (for inspection and tests):
  * which = 0 logits fp32 [T,E], 1 topk_idx int32 [T,k], 2 topk_w fp32 [T,k],
  * 3 offsets int32 [E+1], 4 rows int32 [T*k], 5 pos int32 [T*k],
- * 6 y bf16 [T*k,H], 7 y_shared fp32 [T,H].  Returns (size_t)-1 if invalid. */
+ * 6 y bf16 [T*k,H], 7 y_shared fp32 [T,H], 8 u bf16 [T,H] (the normalised
+ * input of moe_forward_block).  Returns (size_t)-1 if invalid. */
 size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
 
 /* Synchronise `stream`, read and clear the device status word in `ws`.

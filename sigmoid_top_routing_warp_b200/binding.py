@@ -28,13 +28,13 @@ MOE_FLAG_TEST_STALL = 0x1
 STAGE_NAMES = ("router_gemm", "router_select", "dispatch", "gate_up_swiglu", "down_weighted",
                "combine")
 WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "pos": 5,
-            "y": 6, "y_shared": 7}
+            "y": 6, "y_shared": 7, "u": 8}
 
 # Every symbol include/moe.h declares.
 EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
             "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
-            "moe_quantize_act")
+            "moe_quantize_act", "moe_rmsnorm", "moe_forward_block")
 
 
 class MoeConfigC(ctypes.Structure):
@@ -99,6 +99,11 @@ _lib.moe_combine.restype = ctypes.c_int
 _lib.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_forward.restype = ctypes.c_int
 _lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
+_lib.moe_rmsnorm.restype = ctypes.c_int
+_lib.moe_rmsnorm.argtypes = [_CFG, _P, _P, ctypes.c_float, _P, _P]
+_lib.moe_forward_block.restype = ctypes.c_int
+_lib.moe_forward_block.argtypes = ([_CFG, _P, _P, ctypes.c_float] + [_P] * 12 +
+                                   [ctypes.c_size_t, _P, _P])
 _lib.moe_permute_noalloc.restype = ctypes.c_int
 _lib.moe_permute_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_quantize_act.restype = ctypes.c_int
@@ -214,6 +219,29 @@ def moe_forward(cfg, x, w_router, bias, w13, w2, w13s, w2s, out, ws, stream=None
                             ws.numel(), ev, _stream(stream)), "moe_forward")
 
 
+def moe_rmsnorm(cfg, h, gamma, eps, u, stream=None):
+    """Pre-norm of the block input: u = bf16(gamma * h / sqrt(mean(h^2) + eps))."""
+    c = cfg.c()
+    _check(_lib.moe_rmsnorm(ctypes.byref(c), _ptr(h), _ptr(gamma), float(eps), _ptr(u),
+                            _stream(stream)), "moe_rmsnorm")
+
+
+def moe_forward_block(cfg, h, gamma, eps, w_router, bias, w13, w2, w13s, w2s, out, ws,
+                      stream=None, stage_events=None, w13_scale=None, w2_scale=None,
+                      w13s_scale=None, w2s_scale=None):
+    """One pre-norm block: out = h + MoE(RMSNorm(h)); out may be h."""
+    c = cfg.c()
+    ev = None
+    if stage_events is not None:
+        assert len(stage_events) == MOE_NUM_STAGES + 1
+        ev = (ctypes.c_void_p * (MOE_NUM_STAGES + 1))(*[e.cuda_event for e in stage_events])
+    _check(_lib.moe_forward_block(ctypes.byref(c), _ptr(h), _ptr(gamma), float(eps),
+                                  _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w13_scale),
+                                  _ptr(w2), _ptr(w2_scale), _ptr(w13s), _ptr(w13s_scale),
+                                  _ptr(w2s), _ptr(w2s_scale), _ptr(out), _ptr(ws), ws.numel(),
+                                  ev, _stream(stream)), "moe_forward_block")
+
+
 def moe_quantize_act(x, q, scale, stream=None):
     """Step a0 of the FP8 layer: e4m3 codes and per-(row, 128-column) scales."""
     rows, cols = x.shape
@@ -232,7 +260,8 @@ def ws_view(ws: torch.Tensor, cfg: MoeConfig, item: str) -> torch.Tensor:
     shape, dt = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32),
                  "topk_w": ((T, k), torch.float32), "offsets": ((E + 1,), torch.int32),
                  "rows": ((T * k,), torch.int32), "pos": ((T * k,), torch.int32),
-                 "y": ((T * k, H), torch.bfloat16), "y_shared": ((T, H), torch.float32)}[item]
+                 "y": ((T * k, H), torch.bfloat16), "y_shared": ((T, H), torch.float32),
+                 "u": ((T, H), torch.bfloat16)}[item]
     n = 1
     for d in shape:
         n *= d

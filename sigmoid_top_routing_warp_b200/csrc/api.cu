@@ -114,7 +114,7 @@ int router_split(const moe_config_t* c) {
 
 struct Layout {
     size_t status, logits, rpart, idx, w, offsets, rows, pos, wperm, tokstart, chunk, xperm, a, ash,
-        y, ysh, xq, sx, xpq, sxp, aq, sa, ashq, sash, toktiles, total;
+        y, ysh, xq, sx, xpq, sxp, aq, sa, ashq, sash, toktiles, u, total;
 };
 
 Layout layout(const moe_config_t* c) {
@@ -154,6 +154,7 @@ Layout layout(const moe_config_t* c) {
     L.sa = take(q ? n * (I / 128) * 4 : 0);
     L.ashq = take(q ? T * Is : 0);
     L.sash = take(q ? T * (Is / 128) * 4 : 0);
+    L.u = take(T * H * 2);  // normalised block input (moe_forward_block)
     L.total = off;
     return L;
 }
@@ -684,12 +685,33 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
     return MOE_OK;
 }
 
+moe_status_t check_eps(float eps) {
+    if (!(eps >= 0.0f) || !(eps < 1e30f))
+        return fail(MOE_ERR_INVALID_ARG, "eps must be finite and >= 0 (got %g)", (double)eps);
+    return MOE_OK;
+}
+
+moe_status_t run_rmsnorm(const moe_config_t* c, const void* h, const void* gamma, float eps,
+                         void* u, cudaStream_t s) {
+    moe::NormArgs a;
+    a.h = static_cast<const uint16_t*>(h);
+    a.gamma = static_cast<const uint16_t*>(gamma);
+    a.u = static_cast<uint16_t*>(u);
+    a.T = c->T;
+    a.H = c->H;
+    a.eps = eps;
+    MOE_CUDA(moe::launch_rmsnorm(a, s), "rmsnorm launch");
+    return MOE_OK;
+}
+
 moe_status_t run_combine(const moe_config_t* c, const void* y, const int32_t* pos,
-                         const void* y_shared, void* out, cudaStream_t s) {
+                         const void* y_shared, void* out, cudaStream_t s,
+                         const void* residual = nullptr) {
     moe::CombineArgs a;
     a.y = static_cast<const uint16_t*>(y);
     a.pos = pos;
     a.y_shared = static_cast<const float*>(y_shared);
+    a.residual = static_cast<const uint16_t*>(residual);
     a.out = static_cast<uint16_t*>(out);
     a.T = c->T;
     a.k = c->k;
@@ -744,6 +766,7 @@ size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which) {
         case 5: return L.pos;
         case 6: return L.y;
         case 7: return L.ysh;
+        case 8: return L.u;
         default: fail(MOE_ERR_INVALID_ARG, "unknown workspace item %d", which); return (size_t)-1;
     }
 }
@@ -837,17 +860,19 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* 
     return run_combine(cfg, y, pos, y_shared, out, static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_router,
-                         const float* bias, const void* w13, const float* w13_scale,
-                         const void* w2, const float* w2_scale, const void* w13s,
-                         const float* w13s_scale, const void* w2s, const float* w2s_scale,
-                         void* out, void* ws, size_t ws_bytes, void* const* stage_events,
-                         moe_stream_t stream) {
-    g_err[0] = 0;
+// The layer (steps a1-a9) on one stream.  With gamma: the pre-norm block,
+// x is the residual stream h, the layer runs on u = RMSNorm(h) (kept in the
+// workspace) and the combine adds h.
+moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* gamma, float eps,
+                          const void* w_router, const float* bias, const void* w13,
+                          const float* w13_scale, const void* w2, const float* w2_scale,
+                          const void* w13s, const float* w13s_scale, const void* w2s,
+                          const float* w2s_scale, void* out, void* ws, size_t ws_bytes,
+                          void* const* stage_events, moe_stream_t stream) {
     MOE_TRY(check_config(cfg));
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
     MOE_TRY(check_scales(cfg, w13_scale, w2_scale, w13s_scale, w2s_scale));
-    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need16(x, gamma ? "h" : "x"));
     MOE_TRY(need16(w_router, "w_router"));
     MOE_TRY(need(bias, "bias"));
     MOE_TRY(need16(w13, "w13"));
@@ -856,6 +881,10 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
     if (cfg->n_shared > 0) {
         MOE_TRY(need16(w13s, "w13s"));
         MOE_TRY(need16(w2s, "w2s"));
+    }
+    if (gamma) {
+        MOE_TRY(need16(gamma, "gamma"));
+        MOE_TRY(check_eps(eps));
     }
     if (cfg->T == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -878,16 +907,70 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_r
     const int split = router_split(cfg);
     float* gemm_out = split > 1 ? at<float>(ws, L.rpart) : logits;
     MOE_TRY(mark(0));
-    MOE_TRY(run_router_gemm(cfg, x, w_router, gemm_out, at<int>(ws, L.status), s));
+    const void* xin = x;
+    if (gamma) {
+        void* u = at<void>(ws, L.u);
+        MOE_TRY(run_rmsnorm(cfg, x, gamma, eps, u, s));
+        xin = u;
+    }
+    MOE_TRY(run_router_gemm(cfg, xin, w_router, gemm_out, at<int>(ws, L.status), s));
     MOE_TRY(mark(1));
     MOE_TRY(run_select(cfg, gemm_out, bias, idx, w, s, split, logits));
     MOE_TRY(mark(2));
     MOE_TRY(run_permute(cfg, idx, offsets, at<int32_t>(ws, L.rows), pos, ws, s));
     Weights W{w13, w2, w13s, w2s, w13_scale, w2_scale, w13s_scale, w2s_scale};
-    MOE_TRY(run_expert_ffn(cfg, x, offsets, pos, w, W, y, ysh, ws, s, ev[3], ev[4]));
+    MOE_TRY(run_expert_ffn(cfg, xin, offsets, pos, w, W, y, ysh, ws, s, ev[3], ev[4]));
     MOE_TRY(mark(5));
-    MOE_TRY(run_combine(cfg, y, pos, ysh, out, s));
+    MOE_TRY(run_combine(cfg, y, pos, ysh, out, s, gamma ? x : nullptr));
     return mark(6);
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* w_router,
+                         const float* bias, const void* w13, const float* w13_scale,
+                         const void* w2, const float* w2_scale, const void* w13s,
+                         const float* w13s_scale, const void* w2s, const float* w2s_scale,
+                         void* out, void* ws, size_t ws_bytes, void* const* stage_events,
+                         moe_stream_t stream) {
+    g_err[0] = 0;
+    return forward_impl(cfg, x, nullptr, 0.0f, w_router, bias, w13, w13_scale, w2, w2_scale, w13s,
+                        w13s_scale, w2s, w2s_scale, out, ws, ws_bytes, stage_events, stream);
+}
+
+moe_status_t moe_forward_block(const moe_config_t* cfg, const void* h, const void* gamma,
+                               float eps, const void* w_router, const float* bias,
+                               const void* w13, const float* w13_scale, const void* w2,
+                               const float* w2_scale, const void* w13s, const float* w13s_scale,
+                               const void* w2s, const float* w2s_scale, void* out, void* ws,
+                               size_t ws_bytes, void* const* stage_events, moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(need(gamma, "gamma"));
+    if (cfg && h && out && out != h) {
+        const size_t bytes = (size_t)cfg->T * cfg->H * 2;
+        const char* hp = static_cast<const char*>(h);
+        const char* op = static_cast<const char*>(out);
+        if (op < hp + bytes && hp < op + bytes)
+            return fail(MOE_ERR_INVALID_ARG, "out must be h or not overlap it");
+    }
+    return forward_impl(cfg, h, gamma, eps, w_router, bias, w13, w13_scale, w2, w2_scale, w13s,
+                        w13s_scale, w2s, w2s_scale, out, ws, ws_bytes, stage_events, stream);
+}
+
+moe_status_t moe_rmsnorm(const moe_config_t* cfg, const void* h, const void* gamma, float eps,
+                         void* u, moe_stream_t stream) {
+    g_err[0] = 0;
+    if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+    if (cfg->T < 0 || cfg->H <= 0 || cfg->H % 8)
+        return fail(MOE_ERR_INVALID_ARG, "T=%d H=%d: need T >= 0 and H a positive multiple of 8",
+                    cfg->T, cfg->H);
+    MOE_TRY(need16(h, "h"));
+    MOE_TRY(need16(gamma, "gamma"));
+    MOE_TRY(need16(u, "u"));
+    MOE_TRY(check_eps(eps));
+    const size_t bytes = (size_t)cfg->T * cfg->H * 2;
+    const char* hp = static_cast<const char*>(h);
+    const char* up = static_cast<const char*>(u);
+    if (up < hp + bytes && hp < up + bytes) return fail(MOE_ERR_INVALID_ARG, "u must not overlap h");
+    return run_rmsnorm(cfg, h, gamma, eps, u, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_quantize_act(const void* x, int32_t rows, int32_t cols, uint8_t* q, float* scale,

@@ -238,7 +238,8 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// out[t] = bf16( sum_j y[pos[t*k + j]] + y_shared[t] ), 8 columns per thread.
+// out[t] = bf16( sum_j y[pos[t*k + j]] + y_shared[t] (+ residual[t]) ), 8 columns per
+// thread, one fp32 sum in that order and one rounding.
 __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
     const int t = blockIdx.x;
     const int c = blockIdx.y * blockDim.x + threadIdx.x;  // 16-byte chunk
@@ -263,6 +264,16 @@ __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
         const float4 v0 = __ldg(ys), v1 = __ldg(ys + 1);
         acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
         acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+    }
+    if (a.residual) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.residual + (size_t)t * a.H) + c);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+        }
     }
     uint4 o;
     __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);

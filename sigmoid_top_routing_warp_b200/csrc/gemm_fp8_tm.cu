@@ -76,13 +76,32 @@ __device__ __forceinline__ void tm_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// {s, s} as one 64-bit operand of the packed fp32 instructions.
+__device__ __forceinline__ uint64_t tm_splat2(float s) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(s));
+    return r;
+}
+
+// a0 += s * b0, a1 += s * b1 in one packed instruction (two fp32 FMAs, each
+// rounded to nearest: the same bits as two fmaf calls).
+__device__ __forceinline__ void tm_ffma2(float& a0, float& a1, uint64_t ss, uint32_t b0, uint32_t b1) {
+    asm("{\n\t.reg .b64 acc, bb;\n\t"
+        "mov.b64 acc, {%0, %1};\n\t"
+        "mov.b64 bb, {%3, %4};\n\t"
+        "fma.rn.f32x2 acc, %2, bb, acc;\n\t"
+        "mov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "l"(ss), "r"(b0), "r"(b1));
+}
+
 // Promote 16 columns of a partial: acc[j] += s * P[j].
-__device__ __forceinline__ void tm_promote16(uint32_t taddr, float s, float* acc) {
+__device__ __forceinline__ void tm_promote16(uint32_t taddr, uint64_t ss, float* acc) {
     uint32_t r[16];
     tmem_ld_16(taddr, r);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = fmaf(s, __uint_as_float(r[j]), acc[j]);
+    for (int j = 0; j < 16; j += 2) tm_ffma2(acc[j], acc[j + 1], ss, r[j], r[j + 1]);
 }
 
 }  // namespace
@@ -246,22 +265,16 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
             for (int kb0 = 0; kb0 < nk && ok; kb0 += kTMGroup) {
                 if (!wait_bar(&sfull[ss], sph, abort_flag, P.status)) { ok = false; break; }
-                const uint8_t* sl = sring + ss * kTMSSlot;
-                const float4 sx = reinterpret_cast<const float4*>(sl)[tok];
-                const float4 wa = *reinterpret_cast<const float4*>(sl + 2048 + 128 * swa);
-                const float4 wb = *reinterpret_cast<const float4*>(sl + 2048 + 128 * swb);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sempty[ss]);
-                if (++ss == kTMSSlots) { ss = 0; sph ^= 1; }
-                const float sxs[4] = {sx.x, sx.y, sx.z, sx.w};
-                const float was[4] = {wa.x, wa.y, wa.z, wa.w};
-                const float wbs[4] = {wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
+                const float* sl = reinterpret_cast<const float*>(sring + ss * kTMSSlot);
+#pragma unroll 1
                 for (int i = 0; i < kTMGroup; ++i) {
+                    // this K block's scales: the row's s_x and the column halves' s_w
+                    const float sx = sl[4 * tok + i];
+                    const uint64_t sa = tm_splat2(sx * sl[512 + 32 * swa + i]);
+                    const uint64_t sb = tm_splat2(sx * sl[512 + 32 * swb + i]);
                     if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + pb * kTMN;
-                    const float sa = sxs[i] * was[i], sb = sxs[i] * wbs[i];
                     tm_promote16(tb + ca, sa, acc);
                     tm_promote16(tb + ca + 16, sa, acc + 16);
                     tm_promote16(tb + cb, sb, acc + 32);
@@ -271,6 +284,9 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                     if (lane == 0) mbar_arrive(&pempty[pb]);
                     if (++pb == kTMNP) { pb = 0; pph ^= 1; }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sempty[ss]);
+                if (++ss == kTMSSlots) { ss = 0; sph ^= 1; }
             }
             if (!ok) break;
             if (EPI == EPI_SWIGLU) {

@@ -52,10 +52,21 @@ struct CombineArgs {
     const uint16_t* y;        // bf16 [T*k, H]
     const int32_t* pos;       // [T*k]
     const float* y_shared;    // fp32 [T, H] or null
+    const uint16_t* residual; // bf16 [T, H] added in the same fp32 sum, or null
     uint16_t* out;            // bf16 [T, H]
     int T, k, H;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- pre-norm
+struct NormArgs {
+    const uint16_t* h;        // bf16 [T, H]
+    const uint16_t* gamma;    // bf16 [H]
+    uint16_t* u;              // bf16 [T, H]
+    int T, H;                 // H a multiple of 8
+    float eps;
+};
+cudaError_t launch_rmsnorm(const NormArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- FP8 (e4m3, 128-blocks)
 // Activation quantisation: per row, per 128 columns, scale = amax / 448,

@@ -224,3 +224,16 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, seed: int | No
         for key in copies[0]:
             out[key] = [c[key] for c in copies]
     return out
+
+
+# Pre-norm block around the layer: the norm epsilon of the Dots1 config table
+# (rms_norm_eps) and a synthetic norm weight.
+RMS_NORM_EPS = 1e-6
+
+
+def make_norm_weight(wl: Workload, device="cpu", seed: int | None = None) -> torch.Tensor:
+    """RMSNorm weight gamma [H] bf16: 1 + 0.1 N(0, 1), a trained-looking spread
+    around one (seeded separately from the layer's inputs)."""
+    g = _gen(torch.device(device), (wl.seed if seed is None else seed) + 7919)
+    return (1.0 + 0.1 * torch.randn((wl.H,), generator=g, device=device,
+                                    dtype=torch.float32)).to(torch.bfloat16)

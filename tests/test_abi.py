@@ -94,3 +94,41 @@ def test_empty_batch_is_a_no_op(B):
     st = B.lib().moe_forward(ctypes.byref(cc), 16, 16, 16, 16, None, 16, None, 16, None, 16,
                              None, 16, 1 << 20, ws_bytes, None, None)
     assert st == B.MOE_OK
+
+
+def test_block_and_norm_reject_bad_arguments_before_launch(B):
+    c = cfg(B)
+    cc = c.c()
+    ws_bytes = B.workspace_size(c)
+    fake_ws = 1 << 20
+    L = B.lib()
+    st = L.moe_rmsnorm(ctypes.byref(cc), 16, None, ctypes.c_float(1e-6), 1 << 30, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "gamma" in B.get_last_error()
+    st = L.moe_rmsnorm(ctypes.byref(cc), 16, 16, ctypes.c_float(-1.0), 1 << 30, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "eps" in B.get_last_error()
+    st = L.moe_rmsnorm(ctypes.byref(cc), 16, 16, ctypes.c_float(float("nan")), 1 << 30, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "eps" in B.get_last_error()
+    st = L.moe_rmsnorm(ctypes.byref(cc), 1 << 20, 16, ctypes.c_float(1e-6), (1 << 20) + 4096,
+                       None)  # u overlaps h
+    assert st == B.MOE_ERR_INVALID_ARG and "overlap" in B.get_last_error()
+    bad = cfg(B, H=100).c()
+    st = L.moe_rmsnorm(ctypes.byref(bad), 16, 16, ctypes.c_float(1e-6), 1 << 30, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    args = [16] * 12
+    st = L.moe_forward_block(ctypes.byref(cc), 16, None, ctypes.c_float(1e-6), *args, fake_ws,
+                             ws_bytes, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "gamma" in B.get_last_error()
+    st = L.moe_forward_block(ctypes.byref(cc), 1 << 24, 16, ctypes.c_float(1e-6),
+                             16, 16, 16, None, 16, None, 16, None, 16, None, (1 << 24) + 64,
+                             fake_ws, ws_bytes, None, None)  # out partly overlaps h
+    assert st == B.MOE_ERR_INVALID_ARG and "overlap" in B.get_last_error()
+    st = L.moe_forward_block(ctypes.byref(cc), 16, 16, ctypes.c_float(1e-6),
+                             16, 16, 16, None, 16, None, 16, None, 16, None, 16,
+                             fake_ws, ws_bytes - 1, None, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    # empty batch: validated, nothing launched
+    c0 = cfg(B, T=0).c()
+    st = L.moe_forward_block(ctypes.byref(c0), 16, 16, ctypes.c_float(1e-6),
+                             16, 16, 16, None, 16, None, 16, None, 16, None, 16,
+                             fake_ws, B.workspace_size(cfg(B, T=0)), None, None)
+    assert st == B.MOE_OK
