@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--E", type=int, default=None,
                     help="override the routed expert count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the pre-norm block out = h + MoE(RMSNorm(h)) (moe_forward_block)")
     return ap.parse_args()
 
 
@@ -197,6 +199,8 @@ KERNEL_SOURCES = {
     "gate_up_decode": ["csrc/gemm.cu", "csrc/tiles.cuh", "csrc/ptx.cuh", "csrc/kernels.cuh"],
     "gate_up_prefill": ["csrc/gemm_pair.cu", "csrc/ptx.cuh", "csrc/kernels.cuh"],
     "gate_up_fp8": ["csrc/gemm_fp8.cu", "csrc/tiles.cuh", "csrc/ptx.cuh", "csrc/kernels.cuh"],
+    "gate_up_fp8_tm": ["csrc/gemm_fp8_tm.cu", "csrc/tiles.cuh", "csrc/ptx.cuh",
+                       "csrc/kernels.cuh"],
 }
 
 
@@ -282,12 +286,13 @@ def scales_of(inp):
     return {k: inp[k] for k in ("w13_scale", "w2_scale", "w13s_scale", "w2s_scale") if k in inp}
 
 
-def launches_per_step(B, cfg):
+def launches_per_step(B, cfg, block=False):
     from sigmoid_top_routing_warp_b200 import build as _b  # noqa: F401
     permute = 1 if cfg.T * cfg.k <= 4096 else 3
     quant = 1 if cfg.dtype == B.MOE_DTYPE_FP8_E4M3_BLOCK128 else 0
-    # router GEMM, selection, permute, (fp8: quantise x), gather, gate/up GEMM, down GEMM, combine
-    return 2 + permute + quant + 1 + 2 + 1
+    # (block: RMSNorm), router GEMM, selection, permute, (fp8: quantise x), gather,
+    # gate/up GEMM, down GEMM, combine
+    return int(block) + 2 + permute + quant + 1 + 2 + 1
 
 
 def run_ours(args, world, rank, local):
@@ -303,10 +308,21 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     sc = scales_of(inp)
+    gamma = W.make_norm_weight(wl, device=dev, seed=wl.seed + rank) if args.block else None
+    inp["gamma"] = gamma
+
+    def forward(x, events=None):
+        if args.block:  # x is the residual stream h
+            B.moe_forward_block(cfg, x, gamma, W.RMS_NORM_EPS, inp["w_router"], inp["bias"],
+                                inp["w13"], inp["w2"], inp["w13s"], inp["w2s"], out, ws,
+                                stream=stream, stage_events=events, **sc)
+        else:
+            B.moe_forward(cfg, x, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                          inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events,
+                          **sc)
 
     def step(events=None):
-        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                      inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events, **sc)
+        forward(inp["x"], events)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -344,7 +360,7 @@ def run_ours(args, world, rank, local):
     if args.no_e2e:
         return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
                 "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": None,
-                "launches": launches_per_step(B, cfg) * K, "B": B}
+                "launches": launches_per_step(B, cfg, args.block) * K, "B": B}
     # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
     x_host = inp["x"].cpu().pin_memory()
     out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
@@ -352,8 +368,7 @@ def run_ours(args, world, rank, local):
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        B.moe_forward(cfg, x_dev, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                      inp["w13s"], inp["w2s"], out, ws, stream=stream, **sc)
+        forward(x_dev)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -371,13 +386,14 @@ def run_ours(args, world, rank, local):
     barrier(world)
     return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
             "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
-            "launches": launches_per_step(B, cfg) * K, "B": B}
+            "launches": launches_per_step(B, cfg, args.block) * K, "B": B}
 
 
 # ---------------------------------------------------------------- oracle (CPU)
 
 def oracle_sample(wl, inp, seconds: float):
-    """Time the CPU oracle (router logits, selection and layer) on a bounded
+    """Time the CPU oracle (router logits, selection and layer; with a norm
+    weight in inp["gamma"], the pre-norm block around them) on a bounded
     sample of the workload's tokens; returns (tokens/s, threads, sample)."""
     from oracle import oracle as O
 
@@ -405,6 +421,14 @@ def oracle_sample(wl, inp, seconds: float):
     while spent < seconds and rounds < 6:
         toks = rng.choice(wl.T, size=min(n, wl.T), replace=False)
         x = u16(inp["x"][torch.as_tensor(toks, device=inp["x"].device)])
+        gamma = inp.get("gamma")
+        t_norm = 0.0
+        if gamma is not None:  # block: the layer runs on RMSNorm(h)
+            from sigmoid_top_routing_warp_b200 import workloads as W
+            h = x
+            tn = time.perf_counter()
+            x, _ = O.rmsnorm(h, u16(gamma), W.RMS_NORM_EPS)
+            t_norm = time.perf_counter() - tn
         oc = O.Config(T=len(toks), H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
                       n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
                       norm_topk_prob=wl.norm_topk_prob,
@@ -421,10 +445,12 @@ def oracle_sample(wl, inp, seconds: float):
         remap[used] = np.arange(used.size)
         oc2 = O.Config(**{**oc.__dict__, "E": int(used.size)})
         t1 = time.perf_counter()
-        O.layer(oc2, x, remap[idx].astype(np.int32), w, w13, w2, w13s, w2s,
-                w13_scale=wscale("w13_scale", sel), w2_scale=wscale("w2_scale", sel),
-                w13s_scale=wscale("w13s_scale"), w2s_scale=wscale("w2s_scale"))
-        spent += t_route + time.perf_counter() - t1
+        y = O.layer(oc2, x, remap[idx].astype(np.int32), w, w13, w2, w13s, w2s,
+                    w13_scale=wscale("w13_scale", sel), w2_scale=wscale("w2_scale", sel),
+                    w13s_scale=wscale("w13s_scale"), w2s_scale=wscale("w2s_scale"))
+        if gamma is not None:  # residual add
+            y += (h.astype(np.uint32) << 16).view(np.float32)
+        spent += t_norm + t_route + time.perf_counter() - t1
         done += len(toks)
         rounds += 1
         n = min(wl.T, n * 2)
@@ -502,8 +528,12 @@ def main():
                 "frac": ach / pk, "traffic": traffic,
                 "peak_kind": "fp8 sustained (2x measured bf16)" if fp8 else "bf16 sustained",
                 "frac_of_burst_peak": ach / peaks["bf16_tflops"]}
-    kname = ("fp8_gemm_kernel<SWIGLU>" if fp8 else "pair_gemm_kernel<SWIGLU>" if pair else
-             "grouped_gemm_kernel<SWIGLU,16>")
+    tm = fp8 and r["cfg"].T * r["cfg"].k / r["cfg"].E > 48.0 and wl.H % 512 == 0 and wl.I % 512 == 0
+    if tm:
+        kind = "gate_up_fp8_tm"
+        traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
+    kname = ("fp8_tm_gemm_kernel<SWIGLU>" if tm else "fp8_gemm_kernel<SWIGLU>" if fp8 else
+             "pair_gemm_kernel<SWIGLU>" if pair else "grouped_gemm_kernel<SWIGLU,16>")
     roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
                  "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
                  "launch_ms": g1_ms, "peak_source": peak_src})
@@ -524,6 +554,7 @@ def main():
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
                        "I": wl.I, "n_shared": wl.n_shared, "n_group": wl.n_group,
                        "topk_group": wl.topk_group, "experts_touched": r["touched"],
+                       "block": "h + MoE(RMSNorm(h))" if args.block else None,
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
                              % (work["bytes"] / 1e9)},
