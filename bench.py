@@ -505,9 +505,12 @@ def main():
     stage_names = r["B"].STAGE_NAMES
     g1_ms = float(r["stage_ms"][3])
     pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
-    kind = "gate_up_fp8" if wl.dtype == "fp8" else "gate_up_prefill" if pair else "gate_up_decode"
-    traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
     fp8 = wl.dtype == "fp8"
+    # token-major fp8 kernel: more than 48 rows per expert, K dimensions multiples of 512
+    tm = fp8 and r["cfg"].T * r["cfg"].k / r["cfg"].E > 48.0 and wl.H % 512 == 0 and wl.I % 512 == 0
+    kind = ("gate_up_fp8_tm" if tm else "gate_up_fp8" if fp8 else
+            "gate_up_prefill" if pair else "gate_up_decode")
+    traffic = profile_traffic(kind, work["g1_bytes"], wl.name + ("_block" if args.block else ""))
     if fp8:  # the fp8 tensor peak: the measured bf16 peaks x the nominal fp8/bf16 ratio 2
         peaks = dict(peaks)
         for key in ("bf16_tflops", "bf16_tflops_sustained"):
@@ -528,10 +531,6 @@ def main():
                 "frac": ach / pk, "traffic": traffic,
                 "peak_kind": "fp8 sustained (2x measured bf16)" if fp8 else "bf16 sustained",
                 "frac_of_burst_peak": ach / peaks["bf16_tflops"]}
-    tm = fp8 and r["cfg"].T * r["cfg"].k / r["cfg"].E > 48.0 and wl.H % 512 == 0 and wl.I % 512 == 0
-    if tm:
-        kind = "gate_up_fp8_tm"
-        traffic = profile_traffic(kind, work["g1_bytes"], wl.name)
     kname = ("fp8_tm_gemm_kernel<SWIGLU>" if tm else "fp8_gemm_kernel<SWIGLU>" if fp8 else
              "pair_gemm_kernel<SWIGLU>" if pair else "grouped_gemm_kernel<SWIGLU,16>")
     roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
