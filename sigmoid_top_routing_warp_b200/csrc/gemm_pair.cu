@@ -36,7 +36,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kPThreads = 192;
+constexpr int kPThreads = 224;                     // 7 warps
+constexpr int kPTokWarp = 6;                       // token-tile producer
 constexpr int kPBK = 64;
 constexpr int kPHalf = kPairTokens / 2;            // token rows per CTA
 constexpr int kPWBytes = 128 * kPBK * 2;           // 16 KB of weights per CTA
@@ -202,9 +203,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = ptotal<EPI>(P);
 
-    if (warp == 0) {
-        // ---------------------------------------------------- TMA producer (both CTAs)
+    if (warp == 0 || warp == kPTokWarp) {
+        // ---------------------------------------------------- TMA producers (both CTAs)
+        // Warp 0 loads the weight tiles, warp kPTokWarp the token tiles: one
+        // issuing thread tops out near 40 B/clk of 16 KB tensor copies, two
+        // reach the SM's L2 bandwidth.  Both count on the leader's full
+        // barrier; the leader's weight producer sets its expected bytes.
         if (lane == 0) {
+            const bool wprod = warp == 0;
             const uint32_t full_leader = mapa_shared(smem_addr(&full[0]), 0);
             int s = 0;
             uint32_t ph = 0, issued = 0, last_ph = 0;
@@ -222,22 +228,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                     if (!wait_cl(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
                     uint8_t* st = smem + s * kPStage;
                     const uint32_t fb = full_leader + 8u * s;
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
-                    if (EPI == EPI_SWIGLU)
-                        tma_load_5d_pair(st, &p.tw, fb, kb * kPBK, 0, 0, (tl.f0 + 64 * (int)cta) >> 3,
-                                         tl.exp);
-                    else
-                        tma_load_2d_pair(st, &p.tw, fb, kb * kPBK,
-                                         tl.exp * p.n_feat + tl.f0 + 128 * (int)cta);
-                    tma_load_2d_pair(st + kPWBytes, &p.tx[box], fb, kb * kPBK,
-                                     tl.row0 + half * (int)cta);
+                    if (wprod) {
+                        if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
+                        if (EPI == EPI_SWIGLU)
+                            tma_load_5d_pair(st, &p.tw, fb, kb * kPBK, 0, 0,
+                                             (tl.f0 + 64 * (int)cta) >> 3, tl.exp);
+                        else
+                            tma_load_2d_pair(st, &p.tw, fb, kb * kPBK,
+                                             tl.exp * p.n_feat + tl.f0 + 128 * (int)cta);
+                    } else {
+                        tma_load_2d_pair(st + kPWBytes, &p.tx[box], fb, kb * kPBK,
+                                         tl.row0 + half * (int)cta);
+                    }
                     issued |= 1u << s;
                     last_ph = (last_ph & ~(1u << s)) | (ph << s);
                     if (++s == kPStages) { s = 0; ph ^= 1; }
                 }
             }
-            // The leader's full barriers count both CTAs' copies: drain them.
-            if (leader)
+            // The leader's full barriers count both CTAs' copies (weights and
+            // tokens): its weight producer drains them.
+            if (leader && wprod)
                 for (int i = 0; i < kPStages; ++i)
                     if (issued >> i & 1u) wait_cl(&full[i], last_ph >> i & 1u, abort_flag, P.status, true);
         }
