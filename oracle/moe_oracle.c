@@ -522,3 +522,65 @@ void orc_sigmoid_n(const float* x, float* y, int64_t n) {
 void orc_e4m3_encode_n(const float* x, uint8_t* q, int64_t n) {
     for (int64_t i = 0; i < n; ++i) q[i] = orc_f32_to_e4m3(x[i]);
 }
+
+/* ------------------------------------------------------------------------ */
+/* DSA indexer (a second top-k workload next to the layer):                  */
+/*   [DEEP] §4.2 "How DSA Works" and its indexer listing: per index head h, */
+/*   ReLU(q_h . k_h), weighted by a per-query head weight and summed over    */
+/*   heads, then the top-k keys per query;                                   */
+/*   [MLQM] 混合注意力 paragraph: index_topk = 2048 with 64 index heads.      */
+/* Readings: no 1/sqrt(d) scale (the listing has none); an optional causal   */
+/* mask (query t at absolute position q_offset + t sees keys s <= q_offset + */
+/* t); masked scores are -infinity and never selected; the top-k order is    */
+/* score descending, equal scores by lower key index; rows with fewer valid  */
+/* keys than topk are padded with -1.                                        */
+/* q: bf16 [Sq, nh, D]; k: bf16 [Sk, nh, D]; w: bf16 [Sq, nh].               */
+/* ------------------------------------------------------------------------ */
+void orc_dsa_scores(int Sq, int Sk, int nh, int D, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* w, int causal, int q_offset, double* out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < Sq; ++t) {
+        for (int s = 0; s < Sk; ++s) {
+            if (causal && s > q_offset + t) {
+                out[(size_t)t * Sk + s] = -INFINITY;
+                continue;
+            }
+            double acc = 0.0;
+            for (int h = 0; h < nh; ++h) {
+                const uint16_t* qv = q + ((size_t)t * nh + h) * D;
+                const uint16_t* kv = k + ((size_t)s * nh + h) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += (double)orc_bf16_to_f32(qv[d]) * (double)orc_bf16_to_f32(kv[d]);
+                if (dot > 0.0) acc += (double)orc_bf16_to_f32(w[(size_t)t * nh + h]) * dot;
+            }
+            out[(size_t)t * Sk + s] = acc;
+        }
+    }
+}
+
+/* Top-k of each row of binary32 scores [Sq, Sk] -> idx [Sq, topk]: a stable
+ * selection by repeated maximum over the not-yet-chosen keys (plain, O(k Sk)).
+ * -infinity and NaN scores are never chosen. */
+void orc_dsa_topk(int Sq, int Sk, int topk, const float* scores, int32_t* idx) {
+#pragma omp parallel
+    {
+        unsigned char* taken = (unsigned char*)calloc((size_t)Sk, 1);
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < Sq; ++t) {
+            const float* row = scores + (size_t)t * Sk;
+            memset(taken, 0, (size_t)Sk);
+            for (int j = 0; j < topk; ++j) {
+                int best = -1;
+                for (int s = 0; s < Sk; ++s) {
+                    const float v = row[s];
+                    if (taken[s] || !(v > -INFINITY)) continue;  /* skips NaN and -inf */
+                    if (best < 0 || v > row[best]) best = s;       /* strict: lower index wins ties */
+                }
+                idx[(size_t)t * topk + j] = best;
+                if (best >= 0) taken[best] = 1;
+            }
+        }
+        free(taken);
+    }
+}

@@ -100,6 +100,10 @@ def lib():
         _lib.orc_f64_to_bf16_n.argtypes = [P, P, ctypes.c_int64]
         _lib.orc_rmsnorm.restype = None
         _lib.orc_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, P, P, ctypes.c_double, P, P]
+        _lib.orc_dsa_scores.restype = None
+        _lib.orc_dsa_scores.argtypes = [ctypes.c_int] * 4 + [P, P, P, ctypes.c_int, ctypes.c_int, P]
+        _lib.orc_dsa_topk.restype = None
+        _lib.orc_dsa_topk.argtypes = [ctypes.c_int] * 3 + [P, P]
         _lib.orc_set_threads.restype = ctypes.c_int
         _lib.orc_set_threads.argtypes = [ctypes.c_int]
     return _lib
@@ -272,3 +276,28 @@ def block(cfg: Config, h_bf16, gamma_bf16, eps: float, idx, w, w13, w2, w13s, w2
     moe = layer(cfg, u, idx, w, w13, w2, w13s, w2s, tokens=tokens, **scales)
     hv = (h[tokens].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return hv + moe
+
+
+def dsa_scores(q_bf16, k_bf16, w_bf16, causal: bool = False, q_offset: int = 0) -> np.ndarray:
+    """DSA indexer scores I[t, s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,h,:]) in fp64;
+    q [Sq, nh, D], k [Sk, nh, D], w [Sq, nh] as bf16 bits.  Masked entries are -inf."""
+    q = _c(q_bf16, np.uint16)
+    k = _c(k_bf16, np.uint16)
+    w = _c(w_bf16, np.uint16)
+    Sq, nh, D = q.shape
+    Sk = k.shape[0]
+    assert k.shape == (Sk, nh, D) and w.shape == (Sq, nh)
+    out = np.empty((Sq, Sk), dtype=np.float64)
+    lib().orc_dsa_scores(Sq, Sk, nh, D, _p(q), _p(k), _p(w), int(bool(causal)), int(q_offset),
+                         _p(out))
+    return out
+
+
+def dsa_topk(scores_f32, topk: int) -> np.ndarray:
+    """Top-k keys per row of fp32 scores: score descending, equal scores by
+    lower index, -inf never chosen, -1 padding."""
+    sc = _c(scores_f32, np.float32)
+    Sq, Sk = sc.shape
+    idx = np.empty((Sq, topk), dtype=np.int32)
+    lib().orc_dsa_topk(Sq, Sk, int(topk), _p(sc), _p(idx))
+    return idx

@@ -550,3 +550,74 @@ def test_block_is_residual_plus_layer():
     z13, z2 = np.zeros_like(w13), np.zeros_like(w2)
     out0 = O.block(cfg, h, gamma, 1e-6, idx, w, z13, z2, np.zeros_like(w13s), np.zeros_like(w2s))
     np.testing.assert_array_equal(out0, hv)
+
+
+# ---------------------------------------------------------------- DSA indexer
+def _bf16_bits(a):
+    return O.f32_to_bf16(np.asarray(a, dtype=np.float32))
+
+
+def _bits_f64(b):
+    return (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_dsa_scores_against_einsum_and_closed_form():
+    rng = np.random.default_rng(21)
+    Sq, Sk, nh, D = 7, 11, 3, 16
+    q = _bf16_bits(rng.standard_normal((Sq, nh, D)))
+    k = _bf16_bits(rng.standard_normal((Sk, nh, D)))
+    w = _bf16_bits(rng.standard_normal((Sq, nh)))
+    got = O.dsa_scores(q, k, w)
+    dots = np.einsum("thd,shd->tsh", _bits_f64(q), _bits_f64(k))
+    ref = np.einsum("tsh,th->ts", np.maximum(dots, 0.0), _bits_f64(w))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    # one head of width one, unit weight: I[t, s] = max(0, q_t k_s)
+    q1 = _bf16_bits([[[2.0]], [[-1.5]]])
+    k1 = _bf16_bits([[[3.0]], [[-4.0]], [[0.5]]])
+    w1 = _bf16_bits([[1.0], [1.0]])
+    np.testing.assert_array_equal(O.dsa_scores(q1, k1, w1),
+                                  [[6.0, 0.0, 1.0], [0.0, 6.0, 0.0]])
+
+
+def test_dsa_scores_invariants():
+    rng = np.random.default_rng(22)
+    Sq, Sk, nh, D = 5, 9, 4, 8
+    q = _bf16_bits(rng.standard_normal((Sq, nh, D)))
+    k = _bf16_bits(rng.standard_normal((Sk, nh, D)))
+    w = _bf16_bits(rng.standard_normal((Sq, nh)))
+    base = O.dsa_scores(q, k, w)
+    # exact linearity in a power-of-two scale of the head weights
+    w2 = _bf16_bits(_bits_f64(w) * 2.0)
+    np.testing.assert_array_equal(O.dsa_scores(q, k, w2), 2.0 * base)
+    # relabelling the heads (q, k and w together) changes nothing but summation order
+    perm = rng.permutation(nh)
+    np.testing.assert_allclose(O.dsa_scores(q[:, perm], k[:, perm], w[:, perm]), base,
+                               rtol=1e-12, atol=1e-12)
+    # ReLU: keys anti-aligned with every query in head 0 add nothing through head 0
+    kneg = k.copy()
+    kneg[:, 0, :] = _bf16_bits(-np.abs(_bits_f64(k[:, 0, :])))
+    qpos = q.copy()
+    qpos[:, 0, :] = _bf16_bits(np.abs(_bits_f64(q[:, 0, :])))
+    wz = w.copy()
+    wz[:, 0] = 0
+    np.testing.assert_allclose(O.dsa_scores(qpos, kneg, w), O.dsa_scores(qpos, kneg, wz),
+                               rtol=0, atol=0)
+    # causal mask: exactly the keys past each query's absolute position are -inf
+    m = O.dsa_scores(q, k, w, causal=True, q_offset=3)
+    t, s = np.meshgrid(np.arange(Sq), np.arange(Sk), indexing="ij")
+    assert np.isneginf(m[s > t + 3]).all() and np.isfinite(m[s <= t + 3]).all()
+    np.testing.assert_array_equal(m[s <= t + 3], base[s <= t + 3])
+
+
+def test_dsa_topk_against_sorted_brute_force():
+    rng = np.random.default_rng(23)
+    Sq, Sk, topk = 6, 40, 9
+    sc = rng.integers(-3, 4, size=(Sq, Sk)).astype(np.float32)  # many ties
+    sc[0, :35] = -np.inf                                        # 5 valid keys < topk
+    sc[1, 7] = np.nan
+    got = O.dsa_topk(sc, topk)
+    for t in range(Sq):
+        valid = [s for s in range(Sk) if np.isfinite(sc[t, s]) or sc[t, s] == np.inf]
+        order = sorted(valid, key=lambda s: (-float(sc[t, s]), s))[:topk]
+        order += [-1] * (topk - len(order))
+        assert list(got[t]) == order, (t, list(got[t]), order)
