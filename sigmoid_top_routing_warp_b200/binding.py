@@ -34,7 +34,9 @@ WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "p
 EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
             "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
-            "moe_quantize_act", "moe_rmsnorm", "moe_forward_block")
+            "moe_quantize_act", "moe_rmsnorm", "moe_forward_block",
+            "dsa_workspace_size", "dsa_workspace_scores_offset", "dsa_index_scores",
+            "dsa_index_topk", "dsa_indexer")
 
 
 class MoeConfigC(ctypes.Structure):
@@ -99,6 +101,25 @@ _lib.moe_combine.restype = ctypes.c_int
 _lib.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_forward.restype = ctypes.c_int
 _lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
+
+
+class DsaConfigC(ctypes.Structure):
+    _fields_ = [("Sq", ctypes.c_int32), ("Sk", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("q_offset", ctypes.c_int32)]
+
+
+_DCFG = ctypes.POINTER(DsaConfigC)
+_lib.dsa_workspace_size.restype = ctypes.c_size_t
+_lib.dsa_workspace_size.argtypes = [_DCFG]
+_lib.dsa_workspace_scores_offset.restype = ctypes.c_size_t
+_lib.dsa_workspace_scores_offset.argtypes = []
+_lib.dsa_index_scores.restype = ctypes.c_int
+_lib.dsa_index_scores.argtypes = [_DCFG, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.dsa_index_topk.restype = ctypes.c_int
+_lib.dsa_index_topk.argtypes = [_DCFG, _P, _P, _P]
+_lib.dsa_indexer.restype = ctypes.c_int
+_lib.dsa_indexer.argtypes = [_DCFG, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_rmsnorm.restype = ctypes.c_int
 _lib.moe_rmsnorm.argtypes = [_CFG, _P, _P, ctypes.c_float, _P, _P]
 _lib.moe_forward_block.restype = ctypes.c_int
@@ -267,3 +288,55 @@ def ws_view(ws: torch.Tensor, cfg: MoeConfig, item: str) -> torch.Tensor:
         n *= d
     nbytes = n * torch.empty((), dtype=dt).element_size()
     return ws[off:off + nbytes].view(dt).view(shape)
+
+
+# ---------------------------------------------------------------- DSA indexer (include/dsa.h)
+@dataclass
+class DsaConfig:
+    """dsa_config_t: Sq queries, Sk keys, index heads of dim 128, top-k keys."""
+    Sq: int
+    Sk: int
+    n_heads: int = 64
+    head_dim: int = 128
+    topk: int = 2048
+    causal: bool = False
+    q_offset: int = 0
+
+    def c(self) -> DsaConfigC:
+        return DsaConfigC(self.Sq, self.Sk, self.n_heads, self.head_dim, self.topk,
+                          int(bool(self.causal)), self.q_offset)
+
+
+def dsa_workspace_size(cfg: DsaConfig) -> int:
+    c = cfg.c()
+    n = _lib.dsa_workspace_size(ctypes.byref(c))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "dsa_workspace_size")
+    return n
+
+
+def dsa_alloc_workspace(cfg: DsaConfig, device="cuda") -> torch.Tensor:
+    return torch.zeros(dsa_workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def dsa_scores_view(ws: torch.Tensor, cfg: DsaConfig) -> torch.Tensor:
+    off = _lib.dsa_workspace_scores_offset()
+    return ws[off:off + cfg.Sq * cfg.Sk * 4].view(torch.float32).view(cfg.Sq, cfg.Sk)
+
+
+def dsa_index_scores(cfg: DsaConfig, q, k, w, scores, ws, stream=None):
+    c = cfg.c()
+    _check(_lib.dsa_index_scores(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(w), _ptr(scores),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "dsa_index_scores")
+
+
+def dsa_index_topk(cfg: DsaConfig, scores, idx, stream=None):
+    c = cfg.c()
+    _check(_lib.dsa_index_topk(ctypes.byref(c), _ptr(scores), _ptr(idx), _stream(stream)),
+           "dsa_index_topk")
+
+
+def dsa_indexer(cfg: DsaConfig, q, k, w, idx, ws, stream=None):
+    c = cfg.c()
+    _check(_lib.dsa_indexer(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(ws),
+                            ws.numel(), _stream(stream)), "dsa_indexer")

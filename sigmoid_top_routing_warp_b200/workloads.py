@@ -237,3 +237,39 @@ def make_norm_weight(wl: Workload, device="cpu", seed: int | None = None) -> tor
     g = _gen(torch.device(device), (wl.seed if seed is None else seed) + 7919)
     return (1.0 + 0.1 * torch.randn((wl.H,), generator=g, device=device,
                                     dtype=torch.float32)).to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------- DSA indexer inputs
+@dataclass(frozen=True)
+class DsaWorkload:
+    """Indexer scoring + top-k: Sq queries against Sk keys, n_heads index heads
+    of dim 128 (the pages: 64 heads, top-2048)."""
+    name: str
+    Sq: int
+    Sk: int
+    n_heads: int = 64
+    topk: int = 2048
+    causal: bool = True
+    q_offset: int = 0
+    seed: int = 0
+
+
+DSA_WORKLOADS = {
+    "dsa_tiny": DsaWorkload("dsa_tiny", Sq=200, Sk=600, n_heads=8, topk=64, causal=False),
+    # one 8K prefill chunk attending to itself
+    "dsa_prefill": DsaWorkload("dsa_prefill", Sq=8192, Sk=8192),
+    # the last 256 queries of a 64K context
+    "dsa_long": DsaWorkload("dsa_long", Sq=256, Sk=65536, q_offset=65536 - 256),
+}
+
+
+def make_dsa_inputs(wl: DsaWorkload, device="cpu", seed: int | None = None):
+    """q [Sq, nh, 128], k [Sk, nh, 128] ~ N(0, 1) and head weights w [Sq, nh] ~
+    N(0, 1/nh), all bf16 (the projections' outputs; the key norm keeps k at
+    unit scale)."""
+    device = torch.device(device)
+    g = _gen(device, (wl.seed if seed is None else seed) + 4242)
+    D = 128
+    return {"q": _normal_bf16((wl.Sq, wl.n_heads, D), 1.0, g, device),
+            "k": _normal_bf16((wl.Sk, wl.n_heads, D), 1.0, g, device),
+            "w": _normal_bf16((wl.Sq, wl.n_heads), wl.n_heads ** -0.5, g, device)}

@@ -19,9 +19,13 @@ def B():
 
 
 def header_functions():
-    src = open(os.path.join(ROOT, "include", "moe.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b((?:moe|dsa)_[a-z_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(B):
@@ -132,3 +136,28 @@ def test_block_and_norm_reject_bad_arguments_before_launch(B):
                              16, 16, 16, None, 16, None, 16, None, 16, None, 16,
                              fake_ws, B.workspace_size(cfg(B, T=0)), None, None)
     assert st == B.MOE_OK
+
+
+def test_dsa_calls_reject_bad_arguments_before_launch(B):
+    c = B.DsaConfig(Sq=64, Sk=1024)
+    cc = c.c()
+    L = B.lib()
+    n = B.dsa_workspace_size(c)
+    assert n >= 64 * 1024 * 4 and L.dsa_workspace_scores_offset() % 256 == 0
+    for bad in (dict(head_dim=64), dict(topk=0), dict(topk=4096), dict(n_heads=0),
+                dict(Sq=-1), dict(causal=2), dict(q_offset=-3)):
+        kw = dict(Sq=64, Sk=1024)
+        kw.update(bad)
+        with pytest.raises(B.MoeError):
+            B.dsa_workspace_size(B.DsaConfig(**kw))
+    st = L.dsa_index_scores(ctypes.byref(cc), None, 16, 16, 16, 1 << 20, 256, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "q" in B.get_last_error()
+    st = L.dsa_index_scores(ctypes.byref(cc), 24, 16, 16, 16, 1 << 20, 256, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "aligned" in B.get_last_error()
+    st = L.dsa_indexer(ctypes.byref(cc), 16, 16, 16, 16, 1 << 20, n - 1, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    st = L.dsa_index_topk(ctypes.byref(cc), None, 16, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    hd = B.DsaConfig(Sq=4, Sk=4, head_dim=64).c()
+    st = L.dsa_index_topk(ctypes.byref(hd), 16, 16, None)
+    assert st == B.MOE_ERR_UNSUPPORTED
