@@ -145,11 +145,13 @@ def test_dsa_calls_reject_bad_arguments_before_launch(B):
     n = B.dsa_workspace_size(c)
     assert n >= 64 * 1024 * 4 and L.dsa_workspace_scores_offset() % 256 == 0
     for bad in (dict(head_dim=64), dict(topk=0), dict(topk=4096), dict(n_heads=0),
-                dict(Sq=-1), dict(causal=2), dict(q_offset=-3)):
+                dict(Sq=-1), dict(q_offset=-3)):
         kw = dict(Sq=64, Sk=1024)
         kw.update(bad)
         with pytest.raises(B.MoeError):
             B.dsa_workspace_size(B.DsaConfig(**kw))
+    raw = B.DsaConfigC(64, 1024, 64, 128, 2048, 2, 0)  # causal must be 0 or 1
+    assert L.dsa_workspace_size(ctypes.byref(raw)) == 0 and "causal" in B.get_last_error()
     st = L.dsa_index_scores(ctypes.byref(cc), None, 16, 16, 16, 1 << 20, 256, None)
     assert st == B.MOE_ERR_INVALID_ARG and "q" in B.get_last_error()
     st = L.dsa_index_scores(ctypes.byref(cc), 24, 16, 16, 16, 1 << 20, 256, None)
