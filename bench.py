@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--E", type=int, default=None,
                     help="override the routed expert count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dsa-unsorted", action="store_true",
+                    help="DSA workloads: indices by key order (no sort by score)")
     ap.add_argument("--block", action="store_true",
                     help="time the pre-norm block out = h + MoE(RMSNorm(h)) (moe_forward_block)")
     return ap.parse_args()
@@ -463,6 +465,27 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     from sigmoid_top_routing_warp_b200 import workloads as W
+    if args.workload.startswith("dsa_"):
+        wl = W.DSA_WORKLOADS[args.workload]
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        inp = W.make_dsa_inputs(wl, device=dev)
+        per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+        rates = []
+        for i in range(args.warmup + args.steps):
+            r, threads, sample = dsa_oracle_sample(wl, inp, per_step)
+            if i >= args.warmup:
+                rates.append(r)
+        value = float(statistics.median(rates))
+        return {"impl": "reference", "metric": DSA_METRIC, "value": value, "unit": "queries/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": wl.Sq / value * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "Sq": wl.Sq, "Sk": wl.Sk, "n_heads": wl.n_heads,
+                           "topk": wl.topk},
+                "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     wl = W.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.make_inputs(wl, device=dev)
@@ -488,9 +511,169 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- main
 
+# ---------------------------------------------------------------- DSA indexer
+
+DSA_METRIC = "DSA indexer queries/s (scores + top-k) and % roofline (bf16 TFLOP/s), 1×B200"
+
+
+def dsa_work(wl):
+    """Unmasked (query, key) pairs, their MMA FLOPs (2 * heads * 128 each) and
+    the top-k kernel's HBM bytes (scores read once, indices written)."""
+    if wl.causal:
+        lim = np.minimum(wl.q_offset + np.arange(wl.Sq) + 1, wl.Sk)
+        pairs = float(lim.sum())
+    else:
+        pairs = float(wl.Sq) * wl.Sk
+    return {"pairs": pairs, "flops": 2.0 * wl.n_heads * 128 * pairs,
+            "topk_bytes": 4.0 * wl.Sq * wl.Sk + 4.0 * wl.Sq * wl.topk}
+
+
+def dsa_oracle_sample(wl, inp, seconds):
+    from oracle import oracle as O
+
+    def u16(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    threads = O.set_threads(os.cpu_count() or 1)
+    k = u16(inp["k"])
+    rng = np.random.default_rng(3)
+    spent, done, n = 0.0, 0, max(1, threads)
+    while spent < seconds and done < wl.Sq:
+        rows = rng.choice(wl.Sq, size=min(n, wl.Sq), replace=False)
+        for r in rows:
+            q = u16(inp["q"][int(r):int(r) + 1])
+            w = u16(inp["w"][int(r):int(r) + 1])
+            t0 = time.perf_counter()
+            sc = O.dsa_scores(q, k, w, wl.causal, wl.q_offset + int(r))
+            O.dsa_topk(sc.astype(np.float32), wl.topk)
+            spent += time.perf_counter() - t0
+            done += 1
+            if spent >= seconds:
+                break
+        n *= 2
+    return done / spent, threads, "%d query rows of workload %s (%.1f s)" % (done, wl.name, spent)
+
+
+def run_dsa(args, world, rank, local):
+    from sigmoid_top_routing_warp_b200 import binding as B
+    from sigmoid_top_routing_warp_b200 import workloads as W
+
+    wl = W.DSA_WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    inp = W.make_dsa_inputs(wl, device=dev, seed=wl.seed + rank)
+    cfg = B.DsaConfig(Sq=wl.Sq, Sk=wl.Sk, n_heads=wl.n_heads, topk=wl.topk, causal=wl.causal,
+                      q_offset=wl.q_offset, sorted=not args.dsa_unsorted)
+    ws = B.dsa_alloc_workspace(cfg, device=dev)
+    scores = B.dsa_scores_view(ws, cfg)
+    idx = torch.empty((wl.Sq, wl.topk), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        B.dsa_index_scores(cfg, inp["q"], inp["k"], inp["w"], scores, ws, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        B.dsa_index_topk(cfg, scores, idx, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    B.moe_check_device_status(ws)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(dev.index) as clk:
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    B.moe_check_device_status(ws)
+    ms = max_over_ranks(world, t0.elapsed_time(t1))
+    sc_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    tk_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    e2e_ms = None
+    if not args.no_e2e:
+        host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "w")}
+        dev_in = {n: torch.empty_like(inp[n]) for n in ("q", "k", "w")}
+        idx_host = torch.empty((wl.Sq, wl.topk), dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            for n in ("q", "k", "w"):
+                dev_in[n].copy_(host[n], non_blocking=True)
+            B.dsa_indexer(cfg, dev_in["q"], dev_in["k"], dev_in["w"], idx, ws, stream=stream)
+            idx_host.copy_(idx, non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
+    return {"wl": wl, "inp": inp, "ms": ms, "sc_ms": sc_ms, "tk_ms": tk_ms, "clocks": clk.summary(),
+            "e2e_ms": e2e_ms}
+
+
+def dsa_main(args, world, rank, local):
+    peaks, peak_src = load_peaks()
+    r = run_dsa(args, world, rank, local)
+    wl, K = r["wl"], args.steps
+    work = dsa_work(wl)
+    value = world * wl.Sq * K / (r["ms"] / 1e3)
+    ach = work["flops"] / (r["sc_ms"] / 1e3) / 1e12
+    pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tk_gbs = work["topk_bytes"] / (r["tk_ms"] / 1e3) / 1e9
+    line = {"metric": DSA_METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": r["ms"] / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "Sq": wl.Sq, "Sk": wl.Sk, "n_heads": wl.n_heads,
+                       "head_dim": 128, "topk": wl.topk, "causal": wl.causal,
+                       "sorted": not args.dsa_unsorted,
+                       "q_offset": wl.q_offset,
+                       "l2": "inputs larger than L2: %.0f MB of keys and %.0f MB of scores per step"
+                             % (wl.Sk * wl.n_heads * 256 / 1e6, wl.Sq * wl.Sk * 4 / 1e6)},
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                         "frac": ach / pk, "traffic": None, "peak_kind": "bf16 sustained",
+                         "frac_of_burst_peak": ach / peaks["bf16_tflops"],
+                         "kernel": "dsa_scores_kernel (w x ReLU(q.k) over heads)",
+                         "algorithmic_per_launch": work["flops"], "launch_ms": r["sc_ms"],
+                         "peak_source": peak_src},
+            "topk_roofline": {"bound": "hbm", "achieved": tk_gbs, "peak": peaks["hbm_gbs"],
+                              "unit": "GB/s", "frac": tk_gbs / peaks["hbm_gbs"],
+                              "launch_ms": r["tk_ms"]},
+            "stages_ms": {"scores": r["sc_ms"], "topk": r["tk_ms"]},
+            "gpu_launches": 2 * K, "clocks": r["clocks"],
+            "e2e": None if r["e2e_ms"] is None else {
+                "value": world * wl.Sq * K / (r["e2e_ms"] / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": int(sum(r["inp"][n].numel() * 2 for n in ("q", "k", "w"))),
+                "d2h_bytes_per_step": wl.Sq * wl.topk * 4}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, sample = dsa_oracle_sample(wl, r["inp"], args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist_teardown(world)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
+    if args.workload.startswith("dsa_") and args.impl == "ours":
+        dsa_main(args, world, rank, local)
+        return
     if args.impl == "reference":
         line = run_reference(args, world, rank)
         if line is not None:

@@ -11,8 +11,8 @@
  *
  *   I[t, s] = sum_h w[t, h] * max(0, q[t, h, :] . k[s, h, :])
  *   idx[t, :] = the topk keys s of row t with the largest I[t, s], by I
- *               descending, equal scores by lower s first; -1 pads rows with
- *               fewer valid keys.
+ *               descending (or, with sorted = 0, by s ascending), equal
+ *               scores by lower s first; -1 pads rows with fewer valid keys.
  *
  * The projections that make q, k and w (and the key LayerNorm of the
  * listing) are plain per-token GEMMs and norms outside this path.  No 1/sqrt(d)
@@ -40,6 +40,10 @@ typedef struct {
     int32_t topk;      /* keys kept per query (2048 on the pages), 1..2048     */
     int32_t causal;    /* 1: query t sees keys s <= q_offset + t; 0: all keys  */
     int32_t q_offset;  /* absolute position of query 0 (causal only), >= 0     */
+    int32_t sorted;    /* 1: indices by score descending (the listing's        */
+                       /*    torch.topk order); 0: the same set by key index   */
+                       /*    ascending (what a sparse-attention gather needs;  */
+                       /*    skips the sort)                                   */
 } dsa_config_t;
 
 /* Bytes of workspace dsa_index_scores / dsa_indexer need: a 256-byte status

@@ -106,7 +106,7 @@ _lib.moe_forward.argtypes = [_CFG] + [_P] * 13 + [ctypes.c_size_t, _P, _P]
 class DsaConfigC(ctypes.Structure):
     _fields_ = [("Sq", ctypes.c_int32), ("Sk", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("topk", ctypes.c_int32), ("causal", ctypes.c_int32),
-                ("q_offset", ctypes.c_int32)]
+                ("q_offset", ctypes.c_int32), ("sorted", ctypes.c_int32)]
 
 
 _DCFG = ctypes.POINTER(DsaConfigC)
@@ -301,10 +301,11 @@ class DsaConfig:
     topk: int = 2048
     causal: bool = False
     q_offset: int = 0
+    sorted: bool = True      # False: the same set by key index (no sort)
 
     def c(self) -> DsaConfigC:
         return DsaConfigC(self.Sq, self.Sk, self.n_heads, self.head_dim, self.topk,
-                          int(bool(self.causal)), self.q_offset)
+                          int(bool(self.causal)), self.q_offset, int(bool(self.sorted)))
 
 
 def dsa_workspace_size(cfg: DsaConfig) -> int:

@@ -41,6 +41,7 @@ moe_status_t check_cfg(const dsa_config_t* c) {
         return dfail(MOE_ERR_INVALID_ARG, "topk=%lld must be in [1, %lld]", c->topk, moe::kDsaMaxTopk);
     if (c->causal != 0 && c->causal != 1) return dfail(MOE_ERR_INVALID_ARG, "causal must be 0 or 1");
     if (c->q_offset < 0) return dfail(MOE_ERR_INVALID_ARG, "q_offset=%lld must be >= 0", c->q_offset);
+    if (c->sorted != 0 && c->sorted != 1) return dfail(MOE_ERR_INVALID_ARG, "sorted must be 0 or 1");
     return MOE_OK;
 }
 
@@ -100,6 +101,7 @@ moe_status_t run_topk(const dsa_config_t* c, const float* scores, int32_t* idx, 
     a.Sq = c->Sq;
     a.Sk = c->Sk;
     a.topk = c->topk;
+    a.sorted = c->sorted;
     cudaError_t e = moe::launch_dsa_topk(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "DSA top-k kernel launch");
     return MOE_OK;

@@ -6,7 +6,8 @@
 //
 // One CTA per row.  Scores become order-preserving 32-bit keys (a larger
 // float gives a larger key; -inf and NaN give 0, which is never selected).
-// Four 8-bit radix passes (most significant first, shared-memory histograms)
+// Four 8-bit radix passes (most significant first, shared-memory histograms
+// with warp-aggregated counts)
 // find the key T of the k-th largest score.  Every key above T is taken,
 // and of the keys equal to T those with the lowest indices (contiguous
 // per-thread index chunks and block-wide prefix sums keep index order).  The
@@ -96,19 +97,32 @@ __global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs 
         for (int shift = 24; shift >= 0; shift -= 8) {
             for (int b = threadIdx.x; b < 256; b += kTKThreads) hist[b] = 0;
             __syncthreads();
-            for (int s = threadIdx.x; s < Sk; s += kTKThreads) {
-                const uint32_t k = key_at(s);
-                if (k != 0u && (k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+            // warp-aggregated counts: scores cluster in few digits (one
+            // exponent range), so lanes with equal digits add once together
+            for (int s0 = 0; s0 < Sk; s0 += kTKThreads) {
+                const int s = s0 + threadIdx.x;
+                uint32_t k = 0u;
+                if (s < Sk) k = key_at(s);
+                const bool act = k != 0u && (k & mask) == prefix;
+                const uint32_t am = __ballot_sync(0xffffffffu, act);
+                if (act) {
+                    const uint32_t bin = (k >> shift) & 255u;
+                    const uint32_t peers = __match_any_sync(am, bin);
+                    if ((int)(__ffs(peers) - 1) == (threadIdx.x & 31))
+                        atomicAdd(&hist[bin], __popc(peers));
+                }
             }
             __syncthreads();
-            if (threadIdx.x == 0) {
-                int cum = 0, digit = 0;
-                for (int b = 255; b >= 0; --b) {
-                    if (cum + hist[b] >= remaining) { digit = b; break; }
-                    cum += hist[b];
+            // the digit: the highest bin whose suffix count reaches `remaining`
+            // (thread i holds bin 255 - i; an inclusive scan gives suffix counts)
+            {
+                const int hb = threadIdx.x < 256 ? hist[255 - threadIdx.x] : 0;
+                int tot = 0;
+                const int above = block_scan(hb, tmp, &tot);
+                if (threadIdx.x < 256 && above < remaining && above + hb >= remaining) {
+                    sh[0] = 255 - threadIdx.x;
+                    sh[1] = remaining - above;
                 }
-                sh[0] = digit;
-                sh[1] = remaining - cum;
             }
             __syncthreads();
             prefix |= (uint32_t)sh[0] << shift;
@@ -120,30 +134,55 @@ __global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs 
         take_eq = remaining;
     }
 
-    // collect: keys > T anywhere, keys == T by index order up to take_eq
-    const int chunk = (Sk + kTKThreads - 1) / kTKThreads;
-    const int c0 = min(Sk, threadIdx.x * chunk), c1 = min(Sk, c0 + chunk);
+    // collect, in index order: each warp walks its own contiguous segment of
+    // keys with the lanes side by side (coalesced); ballots place each chosen
+    // key.  Keys > T are all taken, keys == T while their rank < take_eq.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int seg = ((Sk + kTKThreads / 32 - 1) / (kTKThreads / 32) + 31) & ~31;
+    const int s_beg = min(Sk, warp * seg), s_end = min(Sk, s_beg + seg);
     int gt = 0, eq = 0;
-    for (int s = c0; s < c1; ++s) {
-        const uint32_t k = key_at(s);
-        gt += k > T;
-        eq += k == T;
+    for (int s0 = s_beg; s0 < s_end; s0 += 32) {
+        const int s = s0 + lane;
+        const uint32_t k = s < s_end ? key_at(s) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, k > T));
+        eq += __popc(__ballot_sync(0xffffffffu, k == T && k != 0u));
     }
     int n_gt = 0, n_eq = 0;
-    const int gt_off = block_scan(gt, tmp, &n_gt);
-    const int eq_off = block_scan(eq, tmp, &n_eq);
+    const int gt_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt : 0, tmp, &n_gt), 0);
+    const int eq_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? eq : 0, tmp, &n_eq), 0);
     (void)n_eq;
-    int pg = gt_off, pe = eq_off;
-    for (int s = c0; s < c1; ++s) {
-        const uint32_t k = key_at(s);
-        const unsigned long long packed =
-            ((unsigned long long)k << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)s);
-        if (k > T) {
-            sortbuf[pg++] = packed;
-        } else if (k == T && k != 0u) {
-            if (pe < take_eq) sortbuf[n_gt + pe] = packed;
-            ++pe;
+    const int eq_take = max(0, min(eq, take_eq - eq_off));
+    int n_sel = 0;
+    const int sel_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt + eq_take : 0, tmp, &n_sel), 0);
+    int32_t* out = a.idx + (size_t)t * a.topk;
+    {
+        int pg = gt_off, pe = eq_off, ps = sel_off;
+        for (int s0 = s_beg; s0 < s_end; s0 += 32) {
+            const int s = s0 + lane;
+            const uint32_t k = s < s_end ? key_at(s) : 0u;
+            const uint32_t bg = __ballot_sync(0xffffffffu, k > T);
+            const uint32_t be = __ballot_sync(0xffffffffu, k == T && k != 0u);
+            const int erank = pe + __popc(be & lt);
+            const bool take_e = ((be >> lane) & 1u) && erank < take_eq;
+            const uint32_t bt = __ballot_sync(0xffffffffu, take_e);
+            if (a.sorted) {
+                const unsigned long long packed =
+                    ((unsigned long long)k << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)s);
+                if ((bg >> lane) & 1u) sortbuf[pg + __popc(bg & lt)] = packed;
+                if (take_e) sortbuf[n_gt + erank] = packed;
+            } else {
+                const uint32_t bsel = bg | bt;
+                if ((bsel >> lane) & 1u) out[ps + __popc(bsel & lt)] = s;
+                ps += __popc(bsel);
+            }
+            pg += __popc(bg);
+            pe += __popc(be);
         }
+    }
+    if (!a.sorted) {
+        for (int j = n_sel + threadIdx.x; j < a.topk; j += kTKThreads) out[j] = -1;
+        return;
     }
     // pad to a power of two with zeros (they sort last) and sort descending
     int P = 32;
@@ -165,7 +204,6 @@ __global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs 
             __syncthreads();
         }
     }
-    int32_t* out = a.idx + (size_t)t * a.topk;
     for (int j = threadIdx.x; j < a.topk; j += kTKThreads)
         out[j] = j < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(sortbuf[j] & 0xFFFFFFFFull)) : -1;
 }

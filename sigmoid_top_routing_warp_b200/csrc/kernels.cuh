@@ -196,6 +196,7 @@ struct DsaTopkArgs {
     int ld;
     int32_t* idx;             // [Sq, topk]
     int Sq, Sk, topk;         // topk <= kDsaMaxTopk
+    int sorted;               // 1: score descending; 0: key index ascending
 };
 size_t dsa_topk_smem(int Sk);
 cudaError_t launch_dsa_topk(const DsaTopkArgs& a, cudaStream_t s);

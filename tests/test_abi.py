@@ -150,7 +150,7 @@ def test_dsa_calls_reject_bad_arguments_before_launch(B):
         kw.update(bad)
         with pytest.raises(B.MoeError):
             B.dsa_workspace_size(B.DsaConfig(**kw))
-    raw = B.DsaConfigC(64, 1024, 64, 128, 2048, 2, 0)  # causal must be 0 or 1
+    raw = B.DsaConfigC(64, 1024, 64, 128, 2048, 2, 0, 1)  # causal must be 0 or 1
     assert L.dsa_workspace_size(ctypes.byref(raw)) == 0 and "causal" in B.get_last_error()
     st = L.dsa_index_scores(ctypes.byref(cc), None, 16, 16, 16, 1 << 20, 256, None)
     assert st == B.MOE_ERR_INVALID_ARG and "q" in B.get_last_error()

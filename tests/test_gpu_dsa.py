@@ -53,6 +53,12 @@ def test_topk_bit_exact(B, Sq, Sk, topk):
     torch.cuda.synchronize()
     ref = O.dsa_topk(sc.cpu().numpy(), topk)
     assert np.array_equal(idx.cpu().numpy(), ref)
+    # index-ordered output: the same set, ascending, -1 padding last
+    B.dsa_index_topk(B.DsaConfig(Sq=Sq, Sk=Sk, n_heads=1, topk=topk, sorted=False), sc, idx)
+    torch.cuda.synchronize()
+    ref_set = np.sort(np.where(ref < 0, np.iinfo(np.int32).max, ref), axis=1)
+    ref_set = np.where(ref_set == np.iinfo(np.int32).max, -1, ref_set)
+    assert np.array_equal(idx.cpu().numpy(), ref_set)
 
 
 def score_bound(q, k, w, rows, causal, q_offset):
