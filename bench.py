@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--E", type=int, default=None,
                     help="override the routed expert count (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="report the eager timed region; by default `value` comes from replays "
+                         "of one captured CUDA graph of the step (stage times and the roofline "
+                         "always come from the eager timed region before it)")
     ap.add_argument("--dsa-unsorted", action="store_true",
                     help="DSA workloads: indices by key order (no sort by score)")
     ap.add_argument("--block", action="store_true",
@@ -313,18 +317,19 @@ def run_ours(args, world, rank, local):
     gamma = W.make_norm_weight(wl, device=dev, seed=wl.seed + rank) if args.block else None
     inp["gamma"] = gamma
 
-    def forward(x, events=None):
+    def forward(x, events=None, st=None):
+        st = stream if st is None else st
         if args.block:  # x is the residual stream h
             B.moe_forward_block(cfg, x, gamma, W.RMS_NORM_EPS, inp["w_router"], inp["bias"],
                                 inp["w13"], inp["w2"], inp["w13s"], inp["w2s"], out, ws,
-                                stream=stream, stage_events=events, **sc)
+                                stream=st, stage_events=events, **sc)
         else:
             B.moe_forward(cfg, x, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                          inp["w13s"], inp["w2s"], out, ws, stream=stream, stage_events=events,
+                          inp["w13s"], inp["w2s"], out, ws, stream=st, stage_events=events,
                           **sc)
 
-    def step(events=None):
-        forward(inp["x"], events)
+    def step(events=None, st=None):
+        forward(inp["x"], events, st)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -359,10 +364,36 @@ def run_ours(args, world, rank, local):
                        for i in range(K)])
     stage_ms = stages.mean(0)
 
+    graph_ms = None
+    if not args.eager:
+        # one step captured on a side stream, replayed K times on it
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gs):
+            with torch.cuda.graph(graph, stream=gs):
+                step(st=gs)
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gs):
+            g0.record(gs)
+            for _ in range(K):
+                graph.replay()
+            g1.record(gs)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        graph_ms = max_over_ranks(world, g0.elapsed_time(g1))
+        B.moe_check_device_status(ws)
+        del graph
     if args.no_e2e:
         return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
                 "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": None,
-                "launches": launches_per_step(B, cfg, args.block) * K, "B": B}
+                "launches": launches_per_step(B, cfg, args.block) * K, "B": B,
+                "graph_ms": graph_ms}
     # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
     x_host = inp["x"].cpu().pin_memory()
     out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
@@ -388,7 +419,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
             "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
-            "launches": launches_per_step(B, cfg, args.block) * K, "B": B}
+            "launches": launches_per_step(B, cfg, args.block) * K, "B": B,
+            "graph_ms": graph_ms}
 
 
 # ---------------------------------------------------------------- oracle (CPU)
@@ -684,7 +716,8 @@ def main():
     r = run_ours(args, world, rank, local)
     wl, K = r["wl"], args.steps
     work = layer_work(wl, r["touched"])
-    value = world * wl.T * K / (r["ms"] / 1e3)
+    step_ms_total = r["graph_ms"] if r["graph_ms"] is not None else r["ms"]
+    value = world * wl.T * K / (step_ms_total / 1e3)
     stage_names = r["B"].STAGE_NAMES
     g1_ms = float(r["stage_ms"][3])
     pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
@@ -719,7 +752,7 @@ def main():
     roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
                  "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
                  "launch_ms": g1_ms, "peak_source": peak_src})
-    layer_ms = r["ms"] / K
+    layer_ms = step_ms_total / K
     tensor_pk = peaks["bf16_tflops"] if hbm_bound else peaks.get("bf16_tflops_sustained",
                                                                      peaks["bf16_tflops"])
     layer = {"ms": layer_ms,
@@ -743,6 +776,8 @@ def main():
             "roofline": roof, "layer_roofline": layer,
             "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
             "gpu_launches": r["launches"], "clocks": r["clocks"],
+            "graph": None if r["graph_ms"] is None else {
+                "ms_per_step": r["graph_ms"] / K, "eager_ms_per_step": r["ms"] / K},
             "e2e": None if r["e2e_ms"] is None else {
                 "value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
