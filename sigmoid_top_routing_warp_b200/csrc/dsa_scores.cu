@@ -211,14 +211,27 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
                     if (!wait_bar(&pfull[pb], pph, abort_flag, a.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + pb * kSK + 64 * g;
+                    uint64_t w2;
+                    asm("mov.b64 %0, {%1, %1};" : "=l"(w2) : "f"(wc));
 #pragma unroll
                     for (int c0 = 0; c0 < 64; c0 += 16) {
                         uint32_t r[16];
                         tmem_ld_16(tb + c0, r);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[c0 + j] = fmaf(wc, fmaxf(__uint_as_float(r[j]), 0.0f), acc[c0 + j]);
+                        for (int j = 0; j < 16; j += 2) {
+                            // acc += w * ReLU(p), two columns per packed FMA (two IEEE
+                            // fp32 FMAs: the same bits as fmaf)
+                            const float p0 = fmaxf(__uint_as_float(r[j]), 0.0f);
+                            const float p1 = fmaxf(__uint_as_float(r[j + 1]), 0.0f);
+                            asm("{\n\t.reg .b64 acc, pp;\n\t"
+                                "mov.b64 acc, {%0, %1};\n\t"
+                                "mov.b64 pp, {%3, %4};\n\t"
+                                "fma.rn.f32x2 acc, %2, pp, acc;\n\t"
+                                "mov.b64 {%0, %1}, acc;\n\t}"
+                                : "+f"(acc[c0 + j]), "+f"(acc[c0 + j + 1])
+                                : "l"(w2), "f"(p0), "f"(p1));
+                        }
                     }
                     tc_fence_before();
                     __syncwarp();
