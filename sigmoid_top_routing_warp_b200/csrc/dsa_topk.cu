@@ -12,7 +12,8 @@
 // and of the keys equal to T those with the lowest indices (contiguous
 // per-thread index chunks and block-wide prefix sums keep index order).  The
 // chosen (key, index) pairs are sorted by key descending, index ascending
-// (one bitonic sort in shared memory) and written as indices; rows with
+// (one bitonic network: steps inside 128-element chunks in registers, the
+// rest in shared memory) and written as indices; rows with
 // fewer valid keys than k are padded with -1.  All decisions are integer
 // comparisons, so equal scores give equal results on any device.
 //
@@ -62,9 +63,69 @@ __device__ __forceinline__ int block_scan(int v, int* tmp, int* total) {
     return before;
 }
 
+__device__ __forceinline__ unsigned long long shfl_xor64(unsigned long long v, int m) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+__device__ __forceinline__ void reg_cmpswap(unsigned long long& x, unsigned long long& y, bool desc) {
+    const unsigned long long hi = x > y ? x : y, lo = x > y ? y : x;
+    x = desc ? hi : lo;
+    y = desc ? lo : hi;
+}
+
+// The descending bitonic network on the 128 elements a warp holds (element
+// base + 4 * lane + r is v[r]).  A pair (lo, lo + stride) of the step for
+// block size `size` is ordered descending when (lo & size) == 0, ascending
+// otherwise: the network of a plain shared-memory bitonic sort, with every
+// step whose partner lies inside the 128-element chunk done in registers.
+// For size >= 8 the bit `size` of an index does not depend on r, so the
+// direction is one flag per lane; strides >= 4 exchange with lane ^ stride/4,
+// strides 2 and 1 stay inside the thread.
+template <int LSTRIDE>
+__device__ __forceinline__ void warp_bitonic_step(unsigned long long (&v)[4], int lane, bool desc) {
+    constexpr int stride = 1 << LSTRIDE;
+    if constexpr (stride >= 4) {
+        const bool keep_max = ((lane & (stride >> 2)) == 0) == desc;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const unsigned long long o = shfl_xor64(v[r], stride >> 2);
+            v[r] = ((v[r] > o) == keep_max) ? v[r] : o;
+        }
+    } else if constexpr (stride == 2) {
+        reg_cmpswap(v[0], v[2], desc);
+        reg_cmpswap(v[1], v[3], desc);
+    } else {
+        reg_cmpswap(v[0], v[1], desc);
+        reg_cmpswap(v[2], v[3], desc);
+    }
+}
+
+// Merge steps of block size 2^LSIZE with strides 2^(LTOP) .. 1, in registers.
+template <int LTOP>
+__device__ __forceinline__ void warp_bitonic_merge(unsigned long long (&v)[4], int lane, bool desc) {
+    warp_bitonic_step<LTOP>(v, lane, desc);
+    if constexpr (LTOP > 0) warp_bitonic_merge<LTOP - 1>(v, lane, desc);
+}
+
+// Sizes 2 .. 128: the chunk ends descending for even base / 128 and
+// ascending for odd (what the first cross-chunk merge needs).
+__device__ __forceinline__ void warp_bitonic_chunk(unsigned long long (&v)[4], int base, int lane) {
+    reg_cmpswap(v[0], v[1], true);   // size 2: pair (4l, 4l+1) descending,
+    reg_cmpswap(v[2], v[3], false);  //         pair (4l+2, 4l+3) ascending
+    const int i0 = base + 4 * lane;
+    warp_bitonic_merge<1>(v, lane, ((i0 >> 2) & 1) == 0);
+    warp_bitonic_merge<2>(v, lane, ((i0 >> 3) & 1) == 0);
+    warp_bitonic_merge<3>(v, lane, ((i0 >> 4) & 1) == 0);
+    warp_bitonic_merge<4>(v, lane, ((i0 >> 5) & 1) == 0);
+    warp_bitonic_merge<5>(v, lane, ((i0 >> 6) & 1) == 0);
+    warp_bitonic_merge<6>(v, lane, ((i0 >> 7) & 1) == 0);
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs a) {
+__global__ void __launch_bounds__(kTKThreads, 4) dsa_topk_kernel(const DsaTopkArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     unsigned long long* sortbuf = reinterpret_cast<unsigned long long*>(smem_raw);  // [kDsaMaxTopk]
     int* hist = reinterpret_cast<int*>(sortbuf + kDsaMaxTopk);                       // [256]
@@ -184,13 +245,26 @@ __global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs 
         for (int j = n_sel + threadIdx.x; j < a.topk; j += kTKThreads) out[j] = -1;
         return;
     }
-    // pad to a power of two with zeros (they sort last) and sort descending
-    int P = 32;
+    // pad to a power of two (>= 128) with zeros (they sort last) and sort
+    // descending: bitonic network, in-chunk steps in registers, the rest in
+    // shared memory
+    int P = 128;
     while (P < want) P <<= 1;
     for (int i = want + threadIdx.x; i < P; i += kTKThreads) sortbuf[i] = 0ull;
     __syncthreads();
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+    const int base = warp * 128;
+    const bool wact = base < P;
+    unsigned long long v[4];
+    if (wact) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) v[r] = sortbuf[base + 4 * lane + r];
+        warp_bitonic_chunk(v, base, lane);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sortbuf[base + 4 * lane + r] = v[r];
+    }
+    __syncthreads();
+    for (int size = 256; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride >= 128; stride >>= 1) {
             for (int i = threadIdx.x; i < P / 2; i += kTKThreads) {
                 const int lo = 2 * i - (i & (stride - 1));
                 const int hi = lo + stride;
@@ -203,6 +277,14 @@ __global__ void __launch_bounds__(kTKThreads) dsa_topk_kernel(const DsaTopkArgs 
             }
             __syncthreads();
         }
+        if (wact) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) v[r] = sortbuf[base + 4 * lane + r];
+            warp_bitonic_merge<6>(v, lane, (base & size) == 0);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sortbuf[base + 4 * lane + r] = v[r];
+        }
+        __syncthreads();
     }
     for (int j = threadIdx.x; j < a.topk; j += kTKThreads)
         out[j] = j < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(sortbuf[j] & 0xFFFFFFFFull)) : -1;
