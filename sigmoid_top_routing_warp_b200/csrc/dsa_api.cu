@@ -2,6 +2,7 @@
 // checks, tensor maps and launches.  Shares the last-error message and the
 // tensor-map helper with api.cu.
 #include "dsa.h"
+#include "dsa_kernels.cuh"
 #include "kernels.cuh"
 
 #include <cuda_runtime.h>
@@ -93,7 +94,10 @@ moe_status_t run_scores(const dsa_config_t* c, const void* q, const void* k, con
     return MOE_OK;
 }
 
-moe_status_t run_topk(const dsa_config_t* c, const float* scores, int32_t* idx, cudaStream_t s) {
+// causal_rows: the scores come from the score kernel, whose causal mask
+// makes keys past q_offset + t -inf in row t, so those are not read.
+moe_status_t run_topk(const dsa_config_t* c, const float* scores, int32_t* idx, bool causal_rows,
+                      cudaStream_t s) {
     moe::DsaTopkArgs a;
     a.scores = scores;
     a.ld = c->Sk;
@@ -102,6 +106,8 @@ moe_status_t run_topk(const dsa_config_t* c, const float* scores, int32_t* idx, 
     a.Sk = c->Sk;
     a.topk = c->topk;
     a.sorted = c->sorted;
+    a.causal = causal_rows && c->causal ? 1 : 0;
+    a.q_offset = c->q_offset;
     cudaError_t e = moe::launch_dsa_topk(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "DSA top-k kernel launch");
     return MOE_OK;
@@ -145,7 +151,7 @@ moe_status_t dsa_index_topk(const dsa_config_t* cfg, const float* scores, int32_
     DSA_TRY(need(scores, "scores", 4));
     DSA_TRY(need(idx, "idx", 4));
     if (cfg->Sq == 0) return MOE_OK;
-    return run_topk(cfg, scores, idx, static_cast<cudaStream_t>(stream));
+    return run_topk(cfg, scores, idx, false, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t dsa_indexer(const dsa_config_t* cfg, const void* q, const void* k, const void* w,
@@ -165,7 +171,7 @@ moe_status_t dsa_indexer(const dsa_config_t* cfg, const void* q, const void* k, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + kDsaStatusBytes);
     if (cfg->Sk > 0) DSA_TRY(run_scores(cfg, q, k, w, scores, ws, s));
-    return run_topk(cfg, scores, idx, s);
+    return run_topk(cfg, scores, idx, true, s);
 }
 
 }  // extern "C"

@@ -27,6 +27,7 @@
 // a group needs stay in L2.
 //
 // Waits are bounded as in the GEMMs (DEV_STATUS_TIMEOUT, abort flag, drain).
+#include "dsa_kernels.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "tiles.cuh"

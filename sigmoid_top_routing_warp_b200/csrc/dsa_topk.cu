@@ -6,20 +6,25 @@
 //
 // One CTA per row.  Scores become order-preserving 32-bit keys (a larger
 // float gives a larger key; -inf and NaN give 0, which is never selected).
-// Four 8-bit radix passes (most significant first, shared-memory histograms
-// with warp-aggregated counts)
-// find the key T of the k-th largest score.  Every key above T is taken,
-// and of the keys equal to T those with the lowest indices (contiguous
-// per-thread index chunks and block-wide prefix sums keep index order).  The
-// chosen (key, index) pairs are sorted by key descending, index ascending
-// (one bitonic network: steps inside 128-element chunks in registers, the
-// rest in shared memory) and written as indices; rows with
-// fewer valid keys than k are padded with -1.  All decisions are integer
-// comparisons, so equal scores give equal results on any device.
+// Four 8-bit radix digits, most significant first, find the key T of the
+// k-th largest score: shared-memory histograms with warp-aggregated counts.
+// The first pass stages the row and counts the top digit; the second keeps
+// the keys of the chosen top digit as candidates (compacted into the sort
+// buffer) and counts their next digit; the last two digits count only the
+// candidates.  Every key above T is taken, and of the keys equal to T those
+// with the lowest indices (per-warp index segments and block-wide prefix
+// sums keep index order).  For sorted output the chosen (key, index) pairs
+// are sorted by key descending, index ascending (one bitonic network: steps
+// inside 128-element chunks in registers, the rest in shared memory); when
+// every key equal to T is taken they are gathered unordered first, since the
+// sort fixes the order.  Rows with fewer valid keys than k are padded with
+// -1.  All decisions are integer comparisons, so equal scores give equal
+// results on any device.  Under a causal mask a row reads only the keys the
+// mask leaves (the others are -inf by construction).
 //
 // Rows of up to kTKCacheKeys scores are staged once in shared memory; longer
-// rows are re-read from global memory on every pass (L2-resident per row).
-#include "kernels.cuh"
+// rows are re-read from global memory (L2-resident per row).
+#include "dsa_kernels.cuh"
 
 namespace moe {
 
@@ -27,6 +32,8 @@ namespace {
 
 constexpr int kTKThreads = 512;
 constexpr int kTKCacheKeys = 32768;    // 128 KB of keys staged in shared memory
+constexpr int kTKCandCap = kDsaMaxTopk * 2;  // candidate keys (uint32) in the sort buffer
+constexpr int kTKBatch = 6;                  // keys loaded per thread before they are used
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -123,105 +130,222 @@ __device__ __forceinline__ void warp_bitonic_chunk(unsigned long long (&v)[4], i
     warp_bitonic_merge<6>(v, lane, ((i0 >> 7) & 1) == 0);
 }
 
+// Adds one to hist[bin] for every lane with `act`: one shared-memory atomic
+// per distinct bin of the warp (scores cluster in few top digits).
+__device__ __forceinline__ void hist_add(bool act, uint32_t bin, int* hist) {
+    const uint32_t am = __ballot_sync(0xffffffffu, act);
+    if (act) {
+        const uint32_t peers = __match_any_sync(am, bin);
+        if ((int)(__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], __popc(peers));
+    }
+}
+
+// The digit of the `remaining`-th largest key: the highest bin whose suffix
+// count reaches it (thread i reads bin 255 - i; an inclusive scan gives
+// suffix counts).  Sets sh[0] = the digit, sh[1] = the rank still wanted
+// inside that bin, sh[2] = the bin's count; returns the sum of all bins.
+// Ends with a barrier, after which sh is valid.
+__device__ __forceinline__ int digit_search(const int* hist, int remaining, int* tmp, int* sh) {
+    const int hb = threadIdx.x < 256 ? hist[255 - threadIdx.x] : 0;
+    int tot = 0;
+    const int above = block_scan(hb, tmp, &tot);
+    if (threadIdx.x < 256 && above < remaining && above + hb >= remaining) {
+        sh[0] = 255 - threadIdx.x;
+        sh[1] = remaining - above;
+        sh[2] = hb;
+    }
+    __syncthreads();
+    return tot;
+}
+
+// Appends the keys of the lanes with `act` at buf[*count ...]: one atomic per
+// warp, order across warps unspecified.  Positions at or past `cap` are not
+// written (the count still grows, so the caller sees the overflow).
+__device__ __forceinline__ void append_key(bool act, uint32_t k, uint32_t* buf, int* count, int cap) {
+    const uint32_t am = __ballot_sync(0xffffffffu, act);
+    if (am == 0u) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(am) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(count, __popc(am));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    const int pos = base + __popc(am & ((1u << lane) - 1u));
+    if (act && pos < cap) buf[pos] = k;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kTKThreads, 4) dsa_topk_kernel(const DsaTopkArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    // sortbuf holds the candidate keys of the radix passes first, then the
+    // chosen (key, index) pairs
     unsigned long long* sortbuf = reinterpret_cast<unsigned long long*>(smem_raw);  // [kDsaMaxTopk]
+    uint32_t* cand = reinterpret_cast<uint32_t*>(sortbuf);                          // [kTKCandCap]
     int* hist = reinterpret_cast<int*>(sortbuf + kDsaMaxTopk);                       // [256]
     int* tmp = hist + 256;                                                           // [32]
-    int* sh = tmp + 32;                                                              // [4]
-    uint32_t* cache = reinterpret_cast<uint32_t*>(sh + 4);                           // [Sk] or none
+    int* sh = tmp + 32;                                                              // [8]
+    uint32_t* cache = reinterpret_cast<uint32_t*>(sh + 8);                           // [Sk] or none
     const int t = blockIdx.x;
     const int Sk = a.Sk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    // keys past the causal limit are the score kernel's -inf: not read
+    const int L = a.causal ? max(0, min(Sk, a.q_offset + t + 1)) : Sk;
     const float* row = a.scores + (size_t)t * a.ld;
     const bool cached = Sk <= kTKCacheKeys;
     auto key_at = [&](int s) -> uint32_t { return cached ? cache[s] : order_key(__ldg(row + s)); };
+    // keys s_first + j * step (j < kTKBatch), 0 at or past `lim`; the loads
+    // are issued before any is used
+    auto load_keys = [&](uint32_t(&kb)[kTKBatch], int s_first, int step, int lim) {
+        if (cached) {
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) {
+                const int s = s_first + j * step;
+                kb[j] = s < lim ? cache[s] : 0u;
+            }
+        } else {
+            float f[kTKBatch];
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) {
+                const int s = s_first + j * step;
+                f[j] = s < lim ? __ldg(row + s) : -INFINITY;
+            }
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) kb[j] = order_key(f[j]);
+        }
+    };
 
-    // stage keys, count valid ones
-    int nv = 0;
-    for (int s = threadIdx.x; s < Sk; s += kTKThreads) {
-        const uint32_t k = order_key(__ldg(row + s));
-        if (cached) cache[s] = k;
-        nv += k != 0u;
+    for (int b = threadIdx.x; b < 256; b += kTKThreads) hist[b] = 0;
+    if (threadIdx.x == 0) sh[3] = sh[4] = 0;
+    __syncthreads();
+    // pass 1: stage the keys, histogram of the top digit (its total counts
+    // the valid keys)
+    // (kTKBatch independent loads in flight per thread before any ballot)
+    for (int s0 = 0; s0 < L; s0 += kTKThreads * kTKBatch) {
+        float f[kTKBatch];
+#pragma unroll
+        for (int j = 0; j < kTKBatch; ++j) {
+            const int s = s0 + j * kTKThreads + threadIdx.x;
+            f[j] = s < L ? __ldg(row + s) : -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < kTKBatch; ++j) {
+            const int s = s0 + j * kTKThreads + threadIdx.x;
+            const uint32_t k = order_key(f[j]);
+            if (cached && s < L) cache[s] = k;
+            hist_add(k != 0u, k >> 24, hist);
+        }
     }
-    int n_valid = 0;
-    block_scan(nv, tmp, &n_valid);   // also a barrier for the cache
+    __syncthreads();
+    const int n_valid = digit_search(hist, a.topk, tmp, sh);
     const int want = min(a.topk, n_valid);
 
-    // threshold key T and how many keys equal to T to take
+    // threshold key T, how many keys equal T (n_eq) and how many of them to
+    // take (take_eq, lowest indices first)
     uint32_t T = 1u;
-    int take_eq = 0;
+    int take_eq = 0, n_eq = 0;
     if (n_valid > a.topk) {
-        uint32_t prefix = 0u, mask = 0u;
-        int remaining = a.topk;
-        for (int shift = 24; shift >= 0; shift -= 8) {
+        uint32_t prefix = (uint32_t)sh[0] << 24, mask = 0xFF000000u;
+        int remaining = sh[1];
+        for (int b = threadIdx.x; b < 256; b += kTKThreads) hist[b] = 0;
+        __syncthreads();
+        // pass 2: the keys of the chosen top digit become candidates;
+        // histogram of their second digit
+        for (int s0 = 0; s0 < L; s0 += kTKThreads * kTKBatch) {
+            uint32_t kb[kTKBatch];
+            load_keys(kb, s0 + threadIdx.x, kTKThreads, L);
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) {
+                const uint32_t k = kb[j];
+                const bool act = k != 0u && (k & mask) == prefix;
+                append_key(act, k, cand, &sh[3], kTKCandCap);
+                hist_add(act, (k >> 16) & 255u, hist);
+            }
+        }
+        __syncthreads();
+        const int n_cand = sh[3];
+        digit_search(hist, remaining, tmp, sh);
+        prefix |= (uint32_t)sh[0] << 16;
+        mask |= 0x00FF0000u;
+        remaining = sh[1];
+        // passes 3 and 4 over the candidates (over the row if they overflowed)
+        const bool from_cand = n_cand <= kTKCandCap;
+        const int n = from_cand ? n_cand : L;
+        for (int shift = 8; shift >= 0; shift -= 8) {
             for (int b = threadIdx.x; b < 256; b += kTKThreads) hist[b] = 0;
             __syncthreads();
-            // warp-aggregated counts: scores cluster in few digits (one
-            // exponent range), so lanes with equal digits add once together
-            for (int s0 = 0; s0 < Sk; s0 += kTKThreads) {
-                const int s = s0 + threadIdx.x;
+            for (int i0 = 0; i0 < n; i0 += kTKThreads) {
+                const int i = i0 + threadIdx.x;
                 uint32_t k = 0u;
-                if (s < Sk) k = key_at(s);
+                if (i < n) k = from_cand ? cand[i] : key_at(i);
                 const bool act = k != 0u && (k & mask) == prefix;
-                const uint32_t am = __ballot_sync(0xffffffffu, act);
-                if (act) {
-                    const uint32_t bin = (k >> shift) & 255u;
-                    const uint32_t peers = __match_any_sync(am, bin);
-                    if ((int)(__ffs(peers) - 1) == (threadIdx.x & 31))
-                        atomicAdd(&hist[bin], __popc(peers));
-                }
+                hist_add(act, (k >> shift) & 255u, hist);
             }
             __syncthreads();
-            // the digit: the highest bin whose suffix count reaches `remaining`
-            // (thread i holds bin 255 - i; an inclusive scan gives suffix counts)
-            {
-                const int hb = threadIdx.x < 256 ? hist[255 - threadIdx.x] : 0;
-                int tot = 0;
-                const int above = block_scan(hb, tmp, &tot);
-                if (threadIdx.x < 256 && above < remaining && above + hb >= remaining) {
-                    sh[0] = 255 - threadIdx.x;
-                    sh[1] = remaining - above;
-                }
-            }
-            __syncthreads();
+            digit_search(hist, remaining, tmp, sh);
             prefix |= (uint32_t)sh[0] << shift;
             mask |= 255u << shift;
             remaining = sh[1];
-            __syncthreads();
+            n_eq = sh[2];
         }
         T = prefix;
         take_eq = remaining;
     }
 
-    // collect, in index order: each warp walks its own contiguous segment of
-    // keys with the lanes side by side (coalesced); ballots place each chosen
-    // key.  Keys > T are all taken, keys == T while their rank < take_eq.
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t lt = (1u << lane) - 1u;
-    const int seg = ((Sk + kTKThreads / 32 - 1) / (kTKThreads / 32) + 31) & ~31;
-    const int s_beg = min(Sk, warp * seg), s_end = min(Sk, s_beg + seg);
-    int gt = 0, eq = 0;
-    for (int s0 = s_beg; s0 < s_end; s0 += 32) {
-        const int s = s0 + lane;
-        const uint32_t k = s < s_end ? key_at(s) : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, k > T));
-        eq += __popc(__ballot_sync(0xffffffffu, k == T && k != 0u));
-    }
-    int n_gt = 0, n_eq = 0;
-    const int gt_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt : 0, tmp, &n_gt), 0);
-    const int eq_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? eq : 0, tmp, &n_eq), 0);
-    (void)n_eq;
-    const int eq_take = max(0, min(eq, take_eq - eq_off));
-    int n_sel = 0;
-    const int sel_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt + eq_take : 0, tmp, &n_sel), 0);
     int32_t* out = a.idx + (size_t)t * a.topk;
-    {
+    int n_sel = want;
+    if (a.sorted && n_eq == take_eq) {
+        // every key >= T is chosen: place the pairs in any order, the sort
+        // below orders them
+        for (int s0 = 0; s0 < L; s0 += kTKThreads * kTKBatch) {
+            uint32_t kb[kTKBatch];
+            load_keys(kb, s0 + threadIdx.x, kTKThreads, L);
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) {
+                const int s = s0 + j * kTKThreads + threadIdx.x;
+                const uint32_t k = kb[j];
+                const bool act = k != 0u && k >= T;
+                const uint32_t am = __ballot_sync(0xffffffffu, act);
+                if (am == 0u) continue;
+                const int leader = __ffs(am) - 1;
+                int base = 0;
+                if (lane == leader) base = atomicAdd(&sh[4], __popc(am));
+                base = __shfl_sync(0xffffffffu, base, leader);
+                if (act)
+                    sortbuf[base + __popc(am & lt)] =
+                        ((unsigned long long)k << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)s);
+            }
+        }
+    } else {
+        // in index order: each warp walks its own contiguous segment of keys
+        // with the lanes side by side (coalesced); ballots place each chosen
+        // key.  Keys > T are all taken, keys == T while their rank < take_eq.
+        const int seg = ((L + kTKThreads / 32 - 1) / (kTKThreads / 32) + 31) & ~31;
+        const int s_beg = min(L, warp * seg), s_end = min(L, s_beg + seg);
+        int gt = 0, eq = 0;
+        for (int s0 = s_beg; s0 < s_end; s0 += 32 * kTKBatch) {
+            uint32_t kb[kTKBatch];
+            load_keys(kb, s0 + lane, 32, s_end);
+#pragma unroll
+            for (int j = 0; j < kTKBatch; ++j) {
+                gt += __popc(__ballot_sync(0xffffffffu, kb[j] > T));
+                eq += __popc(__ballot_sync(0xffffffffu, kb[j] == T && kb[j] != 0u));
+            }
+        }
+        int n_gt = 0, n_eq_all = 0;
+        const int gt_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt : 0, tmp, &n_gt), 0);
+        const int eq_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? eq : 0, tmp, &n_eq_all), 0);
+        (void)n_eq_all;
+        const int eq_take = max(0, min(eq, take_eq - eq_off));
+        const int sel_off = __shfl_sync(0xffffffffu, block_scan(lane == 0 ? gt + eq_take : 0, tmp, &n_sel), 0);
         int pg = gt_off, pe = eq_off, ps = sel_off;
-        for (int s0 = s_beg; s0 < s_end; s0 += 32) {
-            const int s = s0 + lane;
-            const uint32_t k = s < s_end ? key_at(s) : 0u;
+        for (int s0 = s_beg; s0 < s_end; s0 += 32 * kTKBatch) {
+          uint32_t kb[kTKBatch];
+          load_keys(kb, s0 + lane, 32, s_end);
+#pragma unroll
+          for (int j = 0; j < kTKBatch; ++j) {
+            const int s = s0 + 32 * j + lane;
+            const uint32_t k = kb[j];
             const uint32_t bg = __ballot_sync(0xffffffffu, k > T);
             const uint32_t be = __ballot_sync(0xffffffffu, k == T && k != 0u);
             const int erank = pe + __popc(be & lt);
@@ -239,6 +363,7 @@ __global__ void __launch_bounds__(kTKThreads, 4) dsa_topk_kernel(const DsaTopkAr
             }
             pg += __popc(bg);
             pe += __popc(be);
+          }
         }
     }
     if (!a.sorted) {
@@ -291,7 +416,7 @@ __global__ void __launch_bounds__(kTKThreads, 4) dsa_topk_kernel(const DsaTopkAr
 }
 
 size_t dsa_topk_smem(int Sk) {
-    return (size_t)kDsaMaxTopk * 8 + (256 + 32 + 4) * 4 + (Sk <= kTKCacheKeys ? (size_t)Sk * 4 : 0);
+    return (size_t)kDsaMaxTopk * 8 + (256 + 32 + 8) * 4 + (Sk <= kTKCacheKeys ? (size_t)Sk * 4 : 0);
 }
 
 cudaError_t launch_dsa_topk(const DsaTopkArgs& a, cudaStream_t s) {

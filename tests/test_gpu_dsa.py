@@ -61,6 +61,49 @@ def test_topk_bit_exact(B, Sq, Sk, topk):
     assert np.array_equal(idx.cpu().numpy(), ref_set)
 
 
+@pytest.mark.parametrize("Sk,topk,cached", [(20000, 2048, True), (36000, 1000, False)])
+def test_topk_one_top_digit(B, Sk, topk, cached):
+    """Scores in [1, 2) share their top radix digit, so the candidate buffer
+    overflows and the later digits scan the whole row; distinct scores take
+    the unordered gather before the sort; a few duplicated values sit at
+    random places (ties at the threshold go by lower index)."""
+    Sq = 6
+    g = torch.Generator(device="cuda").manual_seed(Sk)
+    sc = 1.0 + torch.rand((Sq, Sk), generator=g, device="cuda")
+    sc[1] = sc[1].sort(descending=True).values  # the k-th largest inside a sorted run
+    sc[2, ::7] = sc[2, 5]                         # one value repeated many times
+    sc[3, : Sk - topk // 2] = float("-inf")       # fewer valid keys than k
+    assert (Sk <= 32768) == cached
+    idx = torch.empty((Sq, topk), dtype=torch.int32, device="cuda")
+    ref = O.dsa_topk(sc.cpu().numpy(), topk)
+    for srt in (True, False):
+        B.dsa_index_topk(B.DsaConfig(Sq=Sq, Sk=Sk, n_heads=1, topk=topk, sorted=srt), sc, idx)
+        torch.cuda.synchronize()
+        want = ref if srt else np.sort(np.where(ref < 0, Sk, ref), axis=1)
+        want = np.where(want == Sk, -1, want)
+        assert np.array_equal(idx.cpu().numpy(), want), srt
+
+
+def test_indexer_causal_small(B, W):
+    """Causal rows with a query offset: each row reads only its unmasked keys
+    (the rest are the score kernel's -inf); selection bit-exact on the GPU's
+    scores, both output orders."""
+    wl = W.DsaWorkload("t", Sq=300, Sk=2500, n_heads=4, topk=256, causal=True, q_offset=2150,
+                       seed=11)
+    inp = W.make_dsa_inputs(wl, device="cuda")
+    for srt in (True, False):
+        cfg = cfg_of(B, wl, sorted=srt)
+        ws = B.dsa_alloc_workspace(cfg)
+        idx = torch.empty((wl.Sq, wl.topk), dtype=torch.int32, device="cuda")
+        B.dsa_indexer(cfg, inp["q"], inp["k"], inp["w"], idx, ws)
+        B.moe_check_device_status(ws)
+        gsc = B.dsa_scores_view(ws, cfg).cpu().numpy()
+        ref = O.dsa_topk(gsc, wl.topk)
+        if not srt:
+            ref = np.sort(ref, axis=1)
+        assert np.array_equal(idx.cpu().numpy(), ref), srt
+
+
 def score_bound(q, k, w, rows, causal, q_offset):
     """|error| bound per entry: 1e-5 * (row max |score| + sum_h |w| |q.k|)."""
     qf = q.float()[rows].double()
