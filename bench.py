@@ -207,6 +207,8 @@ KERNEL_SOURCES = {
     "gate_up_fp8": ["csrc/gemm_fp8.cu", "csrc/tiles.cuh", "csrc/ptx.cuh", "csrc/kernels.cuh"],
     "gate_up_fp8_tm": ["csrc/gemm_fp8_tm.cu", "csrc/tiles.cuh", "csrc/ptx.cuh",
                        "csrc/kernels.cuh"],
+    "dsa_scores": ["csrc/dsa_scores.cu", "csrc/dsa_kernels.cuh", "csrc/kernels.cuh",
+                   "csrc/ptx.cuh", "csrc/tiles.cuh"],
 }
 
 
@@ -227,8 +229,9 @@ def profile_traffic(kind, algorithmic, workload):
     if not os.path.isdir(pdir):
         return None
     ratio = None
+    records = []
     for name in sorted(os.listdir(pdir)):
-        fields = {}
+        # machine-read blocks: each starts with a "kernel:" line
         with open(os.path.join(pdir, name)) as f:
             for line in f:
                 line = line.strip()
@@ -236,7 +239,11 @@ def profile_traffic(kind, algorithmic, workload):
                         "kernel", "traffic_over_algorithmic", "traffic_bytes_per_launch",
                         "source_hash", "workload"):
                     k, v = line.split(":", 1)
-                    fields[k] = v.strip()
+                    if k == "kernel":
+                        records.append({})
+                    if records:
+                        records[-1][k] = v.strip()
+    for fields in records:
         if fields.get("kernel") != kind or fields.get("source_hash") != source_hash(kind):
             continue
         # a capture of this exact workload wins over a ratio scaled from a smaller case
@@ -244,7 +251,7 @@ def profile_traffic(kind, algorithmic, workload):
             return float(fields["traffic_bytes_per_launch"])
         if "traffic_over_algorithmic" in fields and ratio is None:
             ratio = float(fields["traffic_over_algorithmic"])
-    return None if ratio is None else ratio * algorithmic
+    return None if ratio is None or algorithmic is None else ratio * algorithmic
 
 
 # ---------------------------------------------------------------- work model
@@ -677,7 +684,8 @@ def dsa_main(args, world, rank, local):
                        "l2": "inputs larger than L2: %.0f MB of keys and %.0f MB of scores per step"
                              % (wl.Sk * wl.n_heads * 256 / 1e6, wl.Sq * wl.Sk * 4 / 1e6)},
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
-                         "frac": ach / pk, "traffic": None, "peak_kind": "bf16 sustained",
+                         "frac": ach / pk, "traffic": profile_traffic("dsa_scores", None, wl.name),
+                         "peak_kind": "bf16 sustained",
                          "frac_of_burst_peak": ach / peaks["bf16_tflops"],
                          "kernel": "dsa_scores_kernel (w x ReLU(q.k) over heads)",
                          "algorithmic_per_launch": work["flops"], "launch_ms": r["sc_ms"],
