@@ -730,8 +730,8 @@ def main():
     g1_ms = float(r["stage_ms"][3])
     pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
     fp8 = wl.dtype == "fp8"
-    # token-major fp8 kernel: more than 48 rows per expert, K dimensions multiples of 512
-    tm = fp8 and r["cfg"].T * r["cfg"].k / r["cfg"].E > 48.0 and wl.H % 512 == 0 and wl.I % 512 == 0
+    # token-major fp8 kernel: hidden and intermediate sizes multiples of 512
+    tm = fp8 and wl.H % 512 == 0 and wl.I % 512 == 0
     kind = ("gate_up_fp8_tm" if tm else "gate_up_fp8" if fp8 else
             "gate_up_prefill" if pair else "gate_up_decode")
     traffic = profile_traffic(kind, work["g1_bytes"], wl.name + ("_block" if args.block else ""))

@@ -64,14 +64,17 @@ def test_activation_quantisation_bit_exact(B):
 
 SMALL = [
     # name, T, H, E, k, I, n_shared  (weight-major token tiles of 16, 32 and 64,
-    # ragged; H = 768 keeps fp8_tiles64 off the token-major kernel)
+    # ragged: I or H not a multiple of 512 keeps these off the token-major kernel)
     ("fp8_small", 96, 512, 32, 4, 256, 1),
     ("fp8_tiles64", 700, 768, 32, 6, 384, 2),
     ("fp8_tiles32", 200, 512, 32, 6, 256, 1),
     ("fp8_one_token", 1, 512, 32, 8, 128, 1),
-    # token-major kernel (> 48 rows per expert, H and I multiples of 512):
-    # ragged 128-row tiles, experts over two tiles, one K group in the down GEMM
+    # token-major kernel (H and I multiples of 512): ragged 128-row tiles,
+    # experts over two tiles, one K group in the down GEMM, 8 rows per expert,
+    # a single token
     ("fp8_tokmajor", 1200, 1024, 32, 4, 512, 1),
+    ("fp8_tokmajor_sparse", 64, 1024, 32, 4, 512, 1),
+    ("fp8_tokmajor_one_token", 1, 512, 32, 8, 512, 1),
     ("fp8_tokmajor_s2", 700, 1536, 32, 8, 512, 2),
 ]
 
