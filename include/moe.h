@@ -122,7 +122,9 @@ const char* moe_get_last_error(void);
  * (0 if the configuration is invalid; see moe_get_last_error).  The
  * workspace holds logits, routing, the dispatch plan, the gathered
  * activations and the intermediate expert outputs; it must be 256-byte
- * aligned. */
+ * aligned and zero-filled before its first use: its first 256 bytes hold the
+ * status word and the GEMMs' tile-claim counters, which every call leaves at
+ * zero (moe_check_device_status clears the status word). */
 size_t moe_workspace_size(const moe_config_t* cfg);
 
 /* Router: steps a1-a4.  Page: mlqm.cn 稀疏激活 (sigmoid, noaux_tc,

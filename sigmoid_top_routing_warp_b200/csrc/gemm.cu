@@ -17,13 +17,23 @@
 // expert uses bn = 128 token tiles.  The accumulator D[f, r] sits in tensor
 // memory with lane = weight row f and column = token r.
 //
-// Roles (192 threads, one CTA per SM, persistent over a static tile list):
-//   warp 0      TMA producer: weight tile(s) + token tile per 64-wide K step
+// Roles (192 threads, one CTA per SM, persistent):
+//   warp 0      tile claims and TMA producer: weight tile(s) + token tile per
+//               64-wide K step
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //   warps 2..5  epilogue: tcgen05.ld, SiLU*up / x weight / fp32, stores
 // Shared-memory ring of STAGES {weights, tokens} slots with full/empty
 // mbarriers; two TMEM accumulator buffers with full/empty mbarriers so the
 // epilogue of one tile overlaps the main loop of the next.
+//
+// Tiles are claimed at run time: the producer takes the next tile index from
+// a counter in the workspace status block and hands it to the MMA thread and
+// the epilogue through a 4-slot ring.  Claims follow the tile order (expert,
+// feature tile, token tile), so the CTAs working at the same time still
+// share weight tiles in L2, and no CTA sits idle while another has two tiles
+// left: at decode sizes a static round-robin left the CTAs' end times ≈65 µs
+// apart.  The last CTA to finish resets the counter (the workspace starts
+// zero-filled).
 //
 // Every mbarrier wait is bounded: when a wait runs past kWaitLimit cycles the
 // CTA records DEV_STATUS_TIMEOUT in the status word, raises a shared abort
@@ -40,6 +50,8 @@ namespace moe {
 constexpr int kThreads = 192;
 constexpr int kBK = 64;                        // K elements per stage (128 B rows)
 constexpr int kWTileBytes = 128 * kBK * 2;     // one 128-row weight tile
+constexpr int kRing = 4;                       // claimed tile ids in flight (producer -> MMA, epilogue)
+constexpr int kSchedWord = 16;                 // first scheduling word in the status block
 
 template <int BN>
 struct TokTile {
@@ -56,7 +68,7 @@ struct Cfg {
     static constexpr int TMEM_NEED = 2 * ACC_COLS;
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                    : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-    static constexpr int BAR_BYTES = 256;
+    static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16_f32(128, BN);
     static_assert(TMEM_NEED <= 512, "accumulators exceed tensor memory");
@@ -76,7 +88,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* rfull = mma_done + 1;          // [kRing] a claimed tile id is in the ring
+    uint64_t* rempty = rfull + kRing;        // [kRing] read by the MMA thread and 4 epilogue warps
+    int* ring = reinterpret_cast<int*>(rempty + kRing);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,6 +105,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             mbar_init(&tempty[b], 4);
         }
         mbar_init(mma_done, 1);
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 5);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -108,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = total_tiles(P, BN);
+    // tile claim counter and finished-CTA count of this epilogue kind, in the
+    // workspace status block (word 0 is the status word)
+    int* sched = P.status + kSchedWord + 2 * EPI;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -117,7 +139,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             uint32_t issued = 0;          // stages ever filled
             uint32_t last_ph[12] = {0};   // parity of the last fill of each stage
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                // claim the next tile and hand its id to the MMA thread and the epilogue
+                int t = atomicAdd(&sched[0], 1);
+                if (t >= ntiles) t = -1;
+                if (!wait_bar(&rempty[rs], rph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                ring[rs] = t;
+                mbar_arrive(&rfull[rs]);
+                if (++rs == kRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 Tile tl;
                 tile_at(P, BN, t, tl);
                 const GemmProblem& p = P.p[tl.prob];
@@ -153,7 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             int s = 0, buf = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true, any = false;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                if (!wait_bar(&rfull[rs], rph, abort_flag, P.status)) break;
+                const int t = ring[rs];
+                mbar_arrive(&rempty[rs]);
+                if (++rs == kRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 Tile tl;
                 tile_at(P, BN, t, tl);
                 const int nk = P.p[tl.prob].K / kBK / max(P.p[tl.prob].k_split, 1);
@@ -194,7 +233,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const int q = warp & 3;  // tensor-memory lane quadrant of this warp
         int buf = 0;
         uint32_t aph = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        int rs = 0;
+        uint32_t rph = 0;
+        while (true) {
+            if (!wait_bar(&rfull[rs], rph, abort_flag, P.status)) break;
+            const int t = ring[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[rs]);
+            if (++rs == kRing) { rs = 0; rph ^= 1; }
+            if (t < 0) break;
             Tile tl;
             tile_at(P, BN, t, tl);
             const GemmProblem& p = P.p[tl.prob];
@@ -255,6 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+    // the last CTA to finish leaves the claim counters at zero for the next launch
+    // (every CTA's claims came from thread 0 before this point)
+    if (threadIdx.x == 0 && atomicAdd(&sched[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&sched[0], 0);
+        atomicExch(&sched[1], 0);
+    }
 }
 
 template <int EPI, int BN>
@@ -269,6 +322,7 @@ static cudaError_t launch_t(const GemmParams& params, int grid, cudaStream_t s) 
 }
 
 cudaError_t launch_grouped_gemm(int epi, int bn, const GemmParams& params, int grid, cudaStream_t s) {
+    if (params.status == nullptr) return cudaErrorInvalidValue;  // holds the tile claim counters
 #define MOE_GEMM_CASE(E_, B_) \
     if (epi == E_ && bn == B_) return launch_t<E_, B_>(params, grid, s);
     MOE_GEMM_CASE(EPI_F32, 16)

@@ -237,3 +237,24 @@ def test_bounded_wait_timeout_is_reported_and_context_survives(B, W):
     B.moe_check_device_status(ws)
     oidx, ow, _ = O.route(oracle_cfg(cfg), logits.cpu().numpy(), inp["bias"].cpu().numpy())
     assert (idx.cpu().numpy() == oidx).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_tile_claim_counters_reset_and_repeat(B, W, name):
+    """The weight-major GEMMs claim tiles from counters in the workspace status
+    block (words 16..21); every call must leave them at zero, and a second call
+    on the same workspace must produce the same output bit for bit (no tile
+    skipped or done twice)."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl)
+    out1, ws = run_forward(B, cfg, inp)
+    words = ws[:256].view(torch.int32).cpu().numpy()
+    assert (words[16:22] == 0).all(), words[16:22]
+    out2 = torch.empty_like(out1)
+    for _ in range(3):
+        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                      inp.get("w13s"), inp.get("w2s"), out2, ws)
+    B.moe_check_device_status(ws)
+    assert torch.equal(out1, out2)
+    assert (ws[:256].view(torch.int32).cpu().numpy()[16:22] == 0).all()
