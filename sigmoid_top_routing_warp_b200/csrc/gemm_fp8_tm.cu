@@ -32,6 +32,11 @@
 // maxima through shared memory under a bounded mbarrier.
 // EPI_SCALE: y = acc * routing weight, bf16 (or fp32 for the shared expert).
 //
+// Tiles are claimed at run time from a counter in the workspace status block
+// and handed to the MMA thread and the epilogue through a 4-slot ring, as in
+// gemm.cu (with a static round-robin the CTAs' end times spread over 3.5-7.8 %
+// of a launch).
+//
 // Waits are bounded as in gemm.cu (DEV_STATUS_TIMEOUT, abort flag, drain).
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -58,7 +63,9 @@ constexpr int kTMEpiWarps = 16;
 constexpr int kTMThreads = 64 + 32 * kTMEpiWarps;
 constexpr int kTMNP = 2;                       // partial buffers of kTMN columns
 constexpr int kTMAmaxBytes = 2 * 4 * kTMTok * 4;  // [2 parities][4 column groups][128 rows]
-constexpr int kTMBarBytes = 256;
+constexpr int kTMBarBytes = 512;
+constexpr int kTMRing = 4;                     // claimed tile ids in flight (producer -> MMA, epilogue)
+constexpr int kTMSchedWord = 24;               // first scheduling word in the status block
 constexpr int kTMSmem = 1024 + kTMStages * kTMStage + kTMSSlots * kTMSSlot + kTMAmaxBytes +
                         kTMBarBytes;
 // kind::f8f6f4: fp32 accumulator, e4m3 A and B (format 0), K-major, M = 128, N = 256
@@ -127,7 +134,10 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     uint64_t* pempty = pfull + kTMNP;        // partial read (16 epilogue warps)
     uint64_t* amax_bar = pempty + kTMNP;     // [2] row maxima of all column groups written
     uint64_t* mma_done = amax_bar + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* rfull = mma_done + 1;          // [kTMRing] a claimed tile id is in the ring
+    uint64_t* rempty = rfull + kTMRing;      // [kTMRing] read by the MMA thread and the 16 epilogue warps
+    int* ring = reinterpret_cast<int*>(rempty + kTMRing);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kTMRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,6 +156,10 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         }
         for (int b = 0; b < 2; ++b) mbar_init(&amax_bar[b], kTMEpiWarps);
         mbar_init(mma_done, 1);
+        for (int r = 0; r < kTMRing; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 1 + kTMEpiWarps);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -166,6 +180,9 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = total_tiles(P, kTMTok, FSZ);
+    // tile claim counter and finished-CTA count of this epilogue kind (the
+    // workspace status block; word 0 is the status word)
+    int* sched = P.status + kTMSchedWord + 2 * EPI;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -173,7 +190,17 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             int s = 0, ss = 0;
             uint32_t ph = 0, sph = 0, issued = 0, sissued = 0, last_ph = 0, slast_ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                // claim the next tile and hand its id to the MMA thread and the epilogue
+                int t = atomicAdd(&sched[0], 1);
+                if (t >= ntiles) t = -1;
+                if (!wait_bar(&rempty[rs], rph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                ring[rs] = t;
+                mbar_arrive(&rfull[rs]);
+                if (++rs == kTMRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 Tile tl;
                 tile_at(P, kTMTok, t, tl, FSZ);
                 const GemmProblem& p = P.p[tl.prob];
@@ -217,7 +244,14 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             int s = 0, pb = 0;
             uint32_t ph = 0, pph = 0;
             bool ok = true, any = false;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                if (!wait_bar(&rfull[rs], rph, abort_flag, P.status)) break;
+                const int t = ring[rs];
+                mbar_arrive(&rempty[rs]);
+                if (++rs == kTMRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 Tile tl;
                 tile_at(P, kTMTok, t, tl, FSZ);
                 const int nk = P.p[tl.prob].K / kTMBK;
@@ -258,7 +292,15 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         int pb = 0, ss = 0, tile_no = 0;
         uint32_t pph = 0, sph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tile_no) {
+        int rs = 0;
+        uint32_t rph = 0;
+        for (; ok; ++tile_no) {
+            if (!wait_bar(&rfull[rs], rph, abort_flag, P.status)) break;
+            const int t = ring[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[rs]);
+            if (++rs == kTMRing) { rs = 0; rph ^= 1; }
+            if (t < 0) break;
             Tile tl;
             tile_at(P, kTMTok, t, tl, FSZ);
             const GemmProblem& p = P.p[tl.prob];
@@ -369,6 +411,12 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kTMNP * kTMN);
+    // the last CTA to finish leaves the claim counters at zero for the next launch
+    // (every CTA's claims came from thread 0 before this point)
+    if (threadIdx.x == 0 && atomicAdd(&sched[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&sched[0], 0);
+        atomicExch(&sched[1], 0);
+    }
 }
 
 template <int EPI>
@@ -381,6 +429,7 @@ static cudaError_t launch_tm(const GemmParams& params, int grid, cudaStream_t s)
 }
 
 cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cudaStream_t s) {
+    if (params.status == nullptr) return cudaErrorInvalidValue;  // holds the tile claim counters
     if (epi == EPI_SWIGLU) return launch_tm<EPI_SWIGLU>(params, grid, s);
     if (epi == EPI_SCALE) return launch_tm<EPI_SCALE>(params, grid, s);
     return cudaErrorInvalidValue;

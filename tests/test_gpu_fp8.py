@@ -106,3 +106,26 @@ def test_fp8_full_size(B, W, name, sample):
     got = out[torch.as_tensor(toks, device="cuda")].float().cpu().numpy()
     rel = assert_close_fp8(got, ref, name)
     print("%s: rel-L2 %.2e, near-ties %d/%d" % (name, rel, ties, cfg.T))
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[0] in ("fp8_tokmajor", "fp8_tokmajor_sparse")],
+                         ids=lambda c: c[0])
+def test_token_major_claim_counters_reset_and_repeat(B, W, case):
+    """The token-major fp8 GEMMs claim tiles from counters in the workspace
+    status block (words 24..29): a call leaves them at zero, and repeated calls
+    on one workspace give the same output bit for bit."""
+    name, T, H, E, k, I, S = case
+    wl = W.Workload(name, T=T, H=H, E=E, k=k, I=I, n_shared=S, dtype="fp8")
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl)
+    out1, ws = run_forward(B, cfg, inp)
+    assert (ws[:256].view(torch.int32).cpu().numpy()[16:30] == 0).all()
+    out2 = torch.empty_like(out1)
+    for _ in range(3):
+        B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                      inp.get("w13s"), inp.get("w2s"), out2, ws, w13_scale=inp["w13_scale"],
+                      w2_scale=inp["w2_scale"], w13s_scale=inp.get("w13s_scale"),
+                      w2s_scale=inp.get("w2s_scale"))
+    B.moe_check_device_status(ws)
+    assert torch.equal(out1, out2)
+    assert (ws[:256].view(torch.int32).cpu().numpy()[16:30] == 0).all()
