@@ -24,9 +24,11 @@
 // s <= q_offset + t.  Tiles entirely above the diagonal skip loads and MMAs
 // and only store -inf; diagonal tiles store -inf past the limit.  Tiles are
 // walked in groups of 32 query tiles x 4 key tiles so that the q and k rows
-// a group needs stay in L2, and dealt to the CTAs round-robin.  On a causal
-// 8192 x 8192 problem this shape gives the busiest CTA 9 computed tiles
-// (16 x 8 groups gave it 10): the kernel's time follows that maximum.
+// a group needs stay in L2.  CTAs claim tiles at run time in that order from
+// a counter in the workspace status block (the q producer claims and hands
+// the id to the other roles through a 4-slot ring; the last CTA to finish
+// resets the counter): a CTA that drew masked tiles takes more computed ones,
+// so no CTA ends far behind the others.
 //
 // Waits are bounded as in the GEMMs (DEV_STATUS_TIMEOUT, abort flag, drain).
 #include "dsa_kernels.cuh"
@@ -51,7 +53,9 @@ constexpr int kSEpiWarps = 16;
 constexpr int kSBWarp = 2 + kSEpiWarps;        // k-panel producer
 constexpr int kSThreads = 32 * (kSBWarp + 1);
 constexpr int kSNP = 2;
-constexpr int kSBarBytes = 256;
+constexpr int kSBarBytes = 512;
+constexpr int kSRing = 4;                      // claimed tile ids in flight
+constexpr int kSSchedWord = 16;                // first scheduling word in the status block
 constexpr int kSSmem = 1024 + kSStages * kSStage + kSBarBytes;
 constexpr int kSGroupQ = 32, kSGroupK = 4;
 static_assert(kSSmem <= 232448, "shared memory budget");
@@ -92,7 +96,10 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
     uint64_t* pfull = empty + kSStages;
     uint64_t* pempty = pfull + kSNP;
     uint64_t* mma_done = pempty + kSNP;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* rfull = mma_done + 1;          // [kSRing] a claimed tile id is in the ring
+    uint64_t* rempty = rfull + kSRing;       // [kSRing] read by the k producer, the MMA thread, 16 epilogue warps
+    int* ring = reinterpret_cast<int*>(rempty + kSRing);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kSRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -106,6 +113,10 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
             mbar_init(&pempty[b], kSEpiWarps);
         }
         mbar_init(mma_done, 1);
+        for (int r = 0; r < kSRing; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 2 + kSEpiWarps);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -122,6 +133,9 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = ((a.Sq + kSQ - 1) / kSQ) * ((a.Sk + kSK - 1) / kSK);
+    // tile claim counter and finished-CTA count (workspace status block; word 0
+    // is the status word)
+    int* sched = a.status + kSSchedWord;
 
     if (warp == 0 || warp == kSBWarp) {
         // ------------------------------------------------ TMA producers
@@ -130,7 +144,25 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
             int s = 0;
             uint32_t ph = 0, issued = 0, last_ph = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                // the q producer claims the next tile (masked ones too) and hands
+                // its id to the k producer, the MMA thread and the epilogue
+                int t;
+                if (qprod) {
+                    t = atomicAdd(&sched[0], 1);
+                    if (t >= ntiles) t = -1;
+                    if (!wait_bar(&rempty[rs], rph ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ring[rs] = t;
+                    mbar_arrive(&rfull[rs]);
+                } else {
+                    if (!wait_bar(&rfull[rs], rph, abort_flag, a.status)) { ok = false; break; }
+                    t = ring[rs];
+                    mbar_arrive(&rempty[rs]);
+                }
+                if (++rs == kSRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 const STile tl = stile_at(a, t);
                 if (tl.masked) continue;
                 for (int h = 0; h < a.nh && ok; ++h)
@@ -161,7 +193,14 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
             int s = 0, pb = 0;
             uint32_t ph = 0, pph = 0;
             bool ok = true, any = false;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                if (!wait_bar(&rfull[rs], rph, abort_flag, a.status)) break;
+                const int t = ring[rs];
+                mbar_arrive(&rempty[rs]);
+                if (++rs == kSRing) { rs = 0; rph ^= 1; }
+                if (t < 0) break;
                 const STile tl = stile_at(a, t);
                 if (tl.masked) continue;
                 for (int h = 0; h < a.nh && ok; ++h) {
@@ -198,7 +237,15 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
         int pb = 0;
         uint32_t pph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int rs = 0;
+        uint32_t rph = 0;
+        while (ok) {
+            if (!wait_bar(&rfull[rs], rph, abort_flag, a.status)) break;
+            const int t = ring[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[rs]);
+            if (++rs == kSRing) { rs = 0; rph ^= 1; }
+            if (t < 0) break;
             const STile tl = stile_at(a, t);
             const int row = tl.i * kSQ + tok;
             const bool rvalid = row < a.Sq;
@@ -269,6 +316,11 @@ __global__ void __launch_bounds__(kSThreads, 1) dsa_scores_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kSNP * kSK);
+    // the last CTA to finish leaves the claim counters at zero for the next launch
+    if (threadIdx.x == 0 && atomicAdd(&sched[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&sched[0], 0);
+        atomicExch(&sched[1], 0);
+    }
 }
 
 cudaError_t launch_dsa_scores(const DsaScoreArgs& a, int grid, cudaStream_t s) {

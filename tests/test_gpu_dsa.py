@@ -199,3 +199,25 @@ def test_indexer_full_size_sampled(B, W, name, sample):
         tol = 1e-5 * (np.abs(ref[fin]).max() + mag)
         assert (np.abs(gsc[n][fin] - ref[fin]) <= tol[fin]).all()
         check_selection(got[n], ref, 2 * tol, wl.topk)
+
+
+def test_score_claim_counters_reset_and_repeat(B, W):
+    """The score kernel claims tiles from counters in the workspace status
+    block (words 16..17): a call leaves them at zero, and repeated calls on one
+    workspace give the same scores and indices bit for bit."""
+    wl = W.DsaWorkload("t", Sq=700, Sk=1900, n_heads=4, topk=128, causal=True, q_offset=300, seed=3)
+    inp = W.make_dsa_inputs(wl, device="cuda")
+    cfg = cfg_of(B, wl)
+    ws = B.dsa_alloc_workspace(cfg)
+    idx1 = torch.empty((wl.Sq, wl.topk), dtype=torch.int32, device="cuda")
+    B.dsa_indexer(cfg, inp["q"], inp["k"], inp["w"], idx1, ws)
+    B.moe_check_device_status(ws)
+    sc1 = B.dsa_scores_view(ws, cfg).clone()
+    assert (ws[:256].view(torch.int32).cpu().numpy()[16:18] == 0).all()
+    idx2 = torch.empty_like(idx1)
+    for _ in range(3):
+        B.dsa_indexer(cfg, inp["q"], inp["k"], inp["w"], idx2, ws)
+    B.moe_check_device_status(ws)
+    assert torch.equal(sc1.view(torch.int32), B.dsa_scores_view(ws, cfg).view(torch.int32))
+    assert torch.equal(idx1, idx2)
+    assert (ws[:256].view(torch.int32).cpu().numpy()[16:18] == 0).all()
