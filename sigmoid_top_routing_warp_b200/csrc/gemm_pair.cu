@@ -24,6 +24,13 @@
 // warp and row).  Two accumulator buffers (2 x 256 columns) let the epilogue
 // of one tile overlap the main loop of the next.
 //
+// Gate/up tiles are claimed at run time: the leader's weight producer takes the next
+// tile index from a counter in the workspace status block and posts it to
+// both CTAs' 4-slot rings (a remote store and a remote arrive); every role of
+// both CTAs reads it there and releases the slot on the leader.  The last CTA
+// to finish resets the counter (the workspace starts zero-filled).  The down
+// GEMM keeps a static round-robin over the pairs.
+//
 // Every wait is bounded (see wait_cl); on timeout the CTA records
 // DEV_STATUS_TIMEOUT, stops, drains its in-flight copies and MMAs (bounded),
 // meets its peer at the final cluster barrier and frees tensor memory.
@@ -49,6 +56,11 @@ constexpr int kPBarBytes = 256;
 constexpr int kPSmem = 1024 + kPStages * kPStage + kPEpiBytes + kPBarBytes;
 constexpr int kPTmemCols = 2 * kPairTokens;        // two 256-column accumulators
 constexpr long long kPWaitLimit = 1ll << 31;
+constexpr int kPRing = 4;                          // claimed tile ids in flight
+constexpr int kPSchedWord = 32;                    // first scheduling word in the status block
+// consumers of a ring slot: both CTAs' two producers and 4 epilogue warps, and
+// the leader's MMA thread
+constexpr int kPRingReaders = 2 * (2 + 4) + 1;
 static_assert(kPSmem <= 232448, "shared memory budget");
 
 struct PTile {
@@ -152,6 +164,11 @@ __device__ __forceinline__ bool wait_cl(uint64_t* bar, uint32_t parity, volatile
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
+// Store a word into the shared memory of a CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 }  // namespace
 
 template <int EPI>
@@ -166,13 +183,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     uint64_t* tfull = empty + kPStages;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* rfull = mma_done + 1;          // [kPRing] a claimed tile id is in this CTA's ring
+    uint64_t* rempty = rfull + kPRing;       // [kPRing] read by every reader of both CTAs (leader's copy used)
+    int* ring = reinterpret_cast<int*>(rempty + kPRing);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kPRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t cta = cluster_ctarank();
     const bool leader = cta == 0;
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    // gate/up claims tiles at run time; the down GEMM keeps a static
+    // round-robin over the pairs (run-time claims made it ~6 % slower)
+    constexpr bool kClaim = EPI == EPI_SWIGLU;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
@@ -184,6 +207,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             mbar_init(&tempty[b], 8);  // 4 epilogue warps x 2 CTAs (leader's copy used)
         }
         mbar_init(mma_done, 1);
+        for (int r = 0; r < kPRing; ++r) {
+            mbar_init(&rfull[r], 1);                // the leader's claimer
+            mbar_init(&rempty[r], kPRingReaders);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -202,6 +229,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = ptotal<EPI>(P);
+    // tile claim counter and finished-CTA count (workspace status block)
+    int* sched = P.status + kPSchedWord + 2 * EPI;
+    const uint32_t rempty_leader = mapa_shared(smem_addr(&rempty[0]), 0);
+    // the next claimed tile of the pair: waits for its slot, reads the id and
+    // releases the slot on the leader
+    auto next_tile = [&](int& rs, uint32_t& rph, int& t) -> bool {
+        if (!kClaim) {  // rs counts this role's tiles
+            t = pair + rs * npairs;
+            ++rs;
+            if (t >= ntiles) t = -1;
+            return true;
+        }
+        if (!wait_cl(&rfull[rs], rph, abort_flag, P.status)) return false;
+        t = ring[rs];
+        __syncwarp(__activemask());  // every lane has read the id before lane 0 releases it
+        if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(rempty_leader + 8u * rs);
+        if (++rs == kPRing) { rs = 0; rph ^= 1; }
+        return true;
+    };
 
     if (warp == 0 || warp == kPTokWarp) {
         // ---------------------------------------------------- TMA producers (both CTAs)
@@ -215,7 +261,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             int s = 0;
             uint32_t ph = 0, issued = 0, last_ph = 0;
             bool ok = true;
-            for (int t = pair; t < ntiles && ok; t += npairs) {
+            const bool claimer = leader && wprod;
+            const uint32_t ring_peer = mapa_shared(smem_addr(&ring[0]), 1);
+            const uint32_t rfull_peer = mapa_shared(smem_addr(&rfull[0]), 1);
+            int rs = 0, cs = 0;
+            uint32_t rph = 0, cph = 0;
+            while (ok) {
+                if (kClaim && claimer) {
+                    // claim the next tile for the pair and post it to both CTAs
+                    int c = atomicAdd(&sched[0], 1);
+                    if (c >= ntiles) c = -1;
+                    if (!wait_cl(&rempty[cs], cph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    ring[cs] = c;
+                    st_cluster_u32(ring_peer + 4u * cs, (uint32_t)c);
+                    mbar_arrive(&rfull[cs]);
+                    mbar_arrive_cluster(rfull_peer + 8u * cs);
+                    if (++cs == kPRing) { cs = 0; cph ^= 1; }
+                }
+                int t;
+                if (!next_tile(rs, rph, t)) { ok = false; break; }
+                if (t < 0) break;
                 PTile tl;
                 ptile_at<EPI>(P, t, tl);
                 const PairProblem& p = P.p[tl.prob];
@@ -258,7 +323,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             int s = 0, buf = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true, any = false;
-            for (int t = pair; t < ntiles && ok; t += npairs) {
+            int rs = 0;
+            uint32_t rph = 0;
+            while (ok) {
+                int t;
+                if (!next_tile(rs, rph, t) || t < 0) break;
                 PTile tl;
                 ptile_at<EPI>(P, t, tl);
                 const int nk = P.p[tl.prob].K / kPBK;
@@ -296,7 +365,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         uint8_t* stage = epi_buf + q * 4096;
         int buf = 0;
         uint32_t aph = 0;
-        for (int t = pair; t < ntiles; t += npairs) {
+        int rs = 0;
+        uint32_t rph = 0;
+        while (true) {
+            int t;
+            if (!next_tile(rs, rph, t) || t < 0) break;
             PTile tl;
             ptile_at<EPI>(P, t, tl);
             const PairProblem& p = P.p[tl.prob];
@@ -402,6 +475,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem_base, kPTmemCols);
+    // the last CTA to finish leaves the claim counters at zero for the next launch
+    if (kClaim && threadIdx.x == 0 && atomicAdd(&sched[1], 1) == (int)gridDim.x - 1) {
+        atomicExch(&sched[0], 0);
+        atomicExch(&sched[1], 0);
+    }
 }
 
 template <int EPI>
@@ -425,6 +503,7 @@ static cudaError_t launch_pair_t(const PairParams& params, int grid, cudaStream_
 }
 
 cudaError_t launch_pair_gemm(int epi, const PairParams& params, int grid, cudaStream_t s) {
+    if (params.status == nullptr) return cudaErrorInvalidValue;  // holds the tile claim counters
     grid &= ~1;
     if (grid < 2) grid = 2;
     if (epi == EPI_SWIGLU) return launch_pair_t<EPI_SWIGLU>(params, grid, s);
