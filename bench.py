@@ -324,15 +324,16 @@ def run_ours(args, world, rank, local):
     gamma = W.make_norm_weight(wl, device=dev, seed=wl.seed + rank) if args.block else None
     inp["gamma"] = gamma
 
-    def forward(x, events=None, st=None):
+    def forward(x, events=None, st=None, dst=None):
         st = stream if st is None else st
+        dst = out if dst is None else dst
         if args.block:  # x is the residual stream h
             B.moe_forward_block(cfg, x, gamma, W.RMS_NORM_EPS, inp["w_router"], inp["bias"],
-                                inp["w13"], inp["w2"], inp["w13s"], inp["w2s"], out, ws,
+                                inp["w13"], inp["w2"], inp["w13s"], inp["w2s"], dst, ws,
                                 stream=st, stage_events=events, **sc)
         else:
             B.moe_forward(cfg, x, inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
-                          inp["w13s"], inp["w2s"], out, ws, stream=st, stage_events=events,
+                          inp["w13s"], inp["w2s"], dst, ws, stream=st, stage_events=events,
                           **sc)
 
     def step(events=None, st=None):
@@ -401,25 +402,50 @@ def run_ours(args, world, rank, local):
                 "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": None,
                 "launches": launches_per_step(B, cfg, args.block) * K, "B": B,
                 "graph_ms": graph_ms}
-    # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
+    # end to end through the C ABI with host buffers, as a serving loop runs it:
+    # every step copies its x from pinned host memory and its out back, on copy
+    # streams with two device buffers each, so that step i's copies overlap the
+    # neighbouring steps' layer calls (events order every buffer reuse)
     x_host = inp["x"].cpu().pin_memory()
-    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
+    out_host = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
+    out_dev = [torch.empty_like(out) for _ in range(2)]
+    # one stream per direction: an upload never queues behind a read-back that
+    # waits for a layer call
+    up_st, down_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "done", "d2h")}
+    used = [False, False]
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(x_dev)
-        out_host.copy_(out, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(up_st):
+            if used[b]:
+                up_st.wait_event(ev["done"][b])  # step i-2 has read x_dev[b]
+            x_dev[b].copy_(x_host, non_blocking=True)
+            ev["h2d"][b].record(up_st)
+        stream.wait_event(ev["h2d"][b])
+        if used[b]:
+            stream.wait_event(ev["d2h"][b])  # step i-2's out_dev[b] has been read back
+        forward(x_dev[b], dst=out_dev[b])
+        ev["done"][b].record(stream)
+        with torch.cuda.stream(down_st):
+            down_st.wait_event(ev["done"][b])
+            out_host[b].copy_(out_dev[b], non_blocking=True)
+            ev["d2h"][b].record(down_st)
+        used[b] = True
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(K):
-        e2e_step()
+    up_st.wait_stream(stream)
+    down_st.wait_stream(stream)
+    for i in range(K):
+        e2e_step(i)
+    stream.wait_stream(down_st)  # the last read-back is inside the timed region
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
