@@ -666,26 +666,54 @@ def run_dsa(args, world, rank, local):
     tk_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     e2e_ms = None
     if not args.no_e2e:
-        host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "w")}
-        dev_in = {n: torch.empty_like(inp[n]) for n in ("q", "k", "w")}
-        idx_host = torch.empty((wl.Sq, wl.topk), dtype=torch.int32).pin_memory()
+        # the same pipelining as the layer's end-to-end loop: uploads and read-backs on
+        # one copy stream per direction, two device buffers of each, events ordering
+        # every reuse; the scores buffer in the workspace is only touched on `stream`
+        names = ("q", "k", "w")
+        host = {n: inp[n].cpu().pin_memory() for n in names}
+        dev_in = [{n: torch.empty_like(inp[n]) for n in names} for _ in range(2)]
+        idx_dev = [torch.empty_like(idx) for _ in range(2)]
+        idx_host = [torch.empty((wl.Sq, wl.topk), dtype=torch.int32).pin_memory()
+                    for _ in range(2)]
+        up_st, down_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "done", "d2h")}
+        used = [False, False]
 
-        def e2e_step():
-            for n in ("q", "k", "w"):
-                dev_in[n].copy_(host[n], non_blocking=True)
-            B.dsa_indexer(cfg, dev_in["q"], dev_in["k"], dev_in["w"], idx, ws, stream=stream)
-            idx_host.copy_(idx, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            with torch.cuda.stream(up_st):
+                if used[b]:
+                    up_st.wait_event(ev["done"][b])
+                for n in names:
+                    dev_in[b][n].copy_(host[n], non_blocking=True)
+                ev["h2d"][b].record(up_st)
+            stream.wait_event(ev["h2d"][b])
+            if used[b]:
+                stream.wait_event(ev["d2h"][b])
+            B.dsa_indexer(cfg, dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["w"], idx_dev[b], ws,
+                          stream=stream)
+            ev["done"][b].record(stream)
+            with torch.cuda.stream(down_st):
+                down_st.wait_event(ev["done"][b])
+                idx_host[b].copy_(idx_dev[b], non_blocking=True)
+                ev["d2h"][b].record(down_st)
+            used[b] = True
 
-        for _ in range(max(3, args.warmup)):
-            e2e_step()
+        for i in range(max(3, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
+        barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(K):
-            e2e_step()
+        up_st.wait_stream(stream)
+        down_st.wait_stream(stream)
+        for i in range(K):
+            e2e_step(i)
+        stream.wait_stream(down_st)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        B.moe_check_device_status(ws)
         e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
     return {"wl": wl, "inp": inp, "ms": ms, "sc_ms": sc_ms, "tk_ms": tk_ms, "clocks": clk.summary(),
             "e2e_ms": e2e_ms}
