@@ -10,6 +10,7 @@ the Dots1 routing fields with 128 experts, top-6, 2 shared, 1408):
 
   tiny      T=128,   H=512,  E=32,  k=4, I=128,  1 shared
   decode    T=64,    H=5120, E=256, k=8, I=1536, 1 shared, bias U(-0.1,0.1)
+  decode_nobias  the decode shape with a zero bias (near-uniform choice)
   prefill   T=8192,  same shape, bias giving a capped Zipf(1.1) expert load
   fp8_256 / fp8_4096   same shape, e4m3 weights with 128x128 block scales
   grouped   T=16384, H=4096, E=128, k=6, I=1408, 2 shared, n_group=8,
@@ -46,7 +47,7 @@ class Workload:
     norm_topk_prob: bool = True
     routed_scaling_factor: float = 1.0
     dtype: str = "bf16"          # "bf16" | "fp8"
-    bias: str = "uniform"        # "uniform" | "zipf" | "hot"
+    bias: str = "uniform"        # "uniform" | "zero" | "zipf" | "hot"
     seed: int = 0
     x_std: float = 1.0
     w_std: float = 0.02
@@ -62,6 +63,12 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", T=128, H=512, E=32, k=4, I=128),
     "decode": Workload("decode", T=64, H=5120, E=256, k=8, I=1536),
+    # The top-8 sigmoid scores of a decode token lie within ~0.05 of each other
+    # near 1, so a U(-0.1, 0.1) bias largely decides the choice and T=64 tokens
+    # touch ~135-139 experts.  With no bias the choice follows the logits alone
+    # and ~229 of 256 experts are touched: the largest weight stream of a
+    # 64-token batch.
+    "decode_nobias": Workload("decode_nobias", T=64, H=5120, E=256, k=8, I=1536, bias="zero"),
     "prefill": Workload("prefill", T=8192, H=5120, E=256, k=8, I=1536, bias="zipf"),
     "fp8_256": Workload("fp8_256", T=256, H=5120, E=256, k=8, I=1536, dtype="fp8"),
     "fp8_4096": Workload("fp8_4096", T=4096, H=5120, E=256, k=8, I=1536, dtype="fp8"),
@@ -186,6 +193,8 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, seed: int | No
            "w_router": _normal_bf16((E, H), wl.w_std, g, device)}
     if wl.bias == "uniform":
         out["bias"] = (torch.rand((E,), generator=g, device=device) * 0.2 - 0.1).float()
+    elif wl.bias == "zero":
+        out["bias"] = torch.zeros((E,), dtype=torch.float32, device=device)
     else:
         out["bias"] = load_bias_table(bias_table_path(wl)).to(device)
 

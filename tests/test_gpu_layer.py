@@ -207,6 +207,12 @@ def test_full_size_decode(B, W):
     full_size_check(B, W, "decode", sample=6)
 
 
+def test_full_size_decode_nobias(B, W):
+    """The decode shape with a zero bias: ~229 experts touched, one or two rows
+    each, the largest set of segments a 64-token batch has."""
+    full_size_check(B, W, "decode_nobias", sample=6)
+
+
 def test_full_size_prefill_zipf(B, W):
     full_size_check(B, W, "prefill", sample=4)
 

@@ -202,6 +202,26 @@ def test_route_invariants_dots3_shape():
     assert (idx3[clear] == idx[clear]).all()
 
 
+def test_route_zero_bias_is_topk_of_logits_and_bias_concentrates_decode_load():
+    """With b = 0 the choice is the k largest logits (sigmoid is increasing;
+    equal logits by lower index), i.e. a stable argsort.  With the decode
+    batch's U(-0.1, 0.1) bias the same 64 tokens touch far fewer experts: their
+    top-8 sigmoid scores lie close together near 1, so the bias decides."""
+    T, E, k = 64, 256, 8
+    cfg = O.Config(T=T, H=8, E=E, k=k, I=8)
+    for seed in range(3):
+        rng = np.random.default_rng(seed)
+        L = (rng.standard_normal((T, E)) * 1.43).astype(np.float32)
+        b = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+        idx0, w0, _ = O.route(cfg, L, np.zeros(E, np.float32))
+        assert (idx0 == np.argsort(-L, axis=1, kind="stable")[:, :k]).all()
+        idx1, _, _ = O.route(cfg, L, b)
+        touched0, touched1 = len(np.unique(idx0)), len(np.unique(idx1))
+        # a uniform choice of 8 of 256 for 64 tokens touches ~221 on average
+        assert 205 <= touched0 <= 240
+        assert touched1 <= 170
+
+
 def test_route_forced_selection_weights_do_not_see_bias():
     rng = np.random.default_rng(8)
     T, E, k = 64, 32, 4
