@@ -189,7 +189,10 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32_t* topk_id
  *   w2    bf16 [E, H, I]    per expert down projection
  *   w13s  bf16 [2 Is, H]    shared expert gate/up (Is = n_shared * I)
  *   w2s   bf16 [H, Is]      shared expert down
- *   y     bf16 [T*k, H] out w_j * SwiGLU_{idx_j}(x_t) at row pos[t*k + j]
+ *   y     bf16 [T*k, H] out w_j * SwiGLU_{idx_j}(x_t) at row pos[t*k + j];
+ *         fp32 when k == 1: a token's only routed row is then not averaged
+ *         with other experts', and its bf16 rounding alone would be the
+ *         largest error term of the output
  *   y_shared fp32 [T, H] out  SwiGLU_shared(x) (may be NULL iff n_shared == 0);
  *            kept in fp32 because, with weight 1, it is the largest term of
  *            the combine and its rounding would dominate the output error
@@ -220,7 +223,7 @@ moe_status_t moe_quantize_act(const void* x, int32_t rows, int32_t cols, uint8_t
 /* Combine: step a9 (Deep Dive §3.3 "Weighted sum" then shared "add").
  * out_t = sum_{j=0..k-1} y[pos[t*k + j]] + y_shared_t, summed in fp32 in
  * that fixed order (no atomics: bitwise reproducible), rounded once to bf16.
- *   y bf16 [T*k, H], pos int32 [T*k], y_shared fp32 [T, H] or NULL,
+ *   y bf16 [T*k, H] (fp32 when k == 1), pos int32 [T*k], y_shared fp32 [T, H] or NULL,
  *   out bf16 [T, H]                                                        */
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* pos,
                          const void* y_shared, void* out, moe_stream_t stream);
@@ -271,7 +274,7 @@ moe_status_t moe_forward_block(const moe_config_t* cfg, const void* h, const voi
  * moe_forward leaves there (for inspection and tests):
  * which = 0 logits fp32 [T,E], 1 topk_idx int32 [T,k], 2 topk_w fp32 [T,k],
  * 3 offsets int32 [E+1], 4 rows int32 [T*k], 5 pos int32 [T*k],
- * 6 y bf16 [T*k,H], 7 y_shared fp32 [T,H], 8 u bf16 [T,H] (the normalised
+ * 6 y bf16 [T*k,H] (fp32 when k == 1), 7 y_shared fp32 [T,H], 8 u bf16 [T,H] (the normalised
  * input of moe_forward_block).  Returns (size_t)-1 if invalid. */
 size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
 

@@ -281,7 +281,8 @@ def ws_view(ws: torch.Tensor, cfg: MoeConfig, item: str) -> torch.Tensor:
     shape, dt = {"logits": ((T, E), torch.float32), "topk_idx": ((T, k), torch.int32),
                  "topk_w": ((T, k), torch.float32), "offsets": ((E + 1,), torch.int32),
                  "rows": ((T * k,), torch.int32), "pos": ((T * k,), torch.int32),
-                 "y": ((T * k, H), torch.bfloat16), "y_shared": ((T, H), torch.float32),
+                 "y": ((T * k, H), torch.float32 if k == 1 else torch.bfloat16),
+                 "y_shared": ((T, H), torch.float32),
                  "u": ((T, H), torch.bfloat16)}[item]
     n = 1
     for d in shape:

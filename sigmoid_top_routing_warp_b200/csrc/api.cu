@@ -149,7 +149,7 @@ Layout layout(const moe_config_t* c) {
     L.xperm = take(n * H * 2);
     L.a = take(n * I * 2);
     L.ash = take(T * Is * 2);
-    L.y = take(n * H * 2);
+    L.y = take(n * H * (c->k == 1 ? 4 : 2));  // routed outputs: fp32 when k = 1
     L.ysh = take(T * H * 4);
     const bool q = is_fp8(c);
     L.xq = take(q ? T * H : 0);
@@ -480,6 +480,7 @@ moe_status_t run_expert_ffn_fp8(const moe_config_t* c, const void* x, const int3
         p.out = y;
         p.ld_out = c->H;
         p.row_w = g.w_perm;
+        p.out_f32 = c->k == 1;
         p.w_scale = W.s2;
         p.x_scale = at<float>(ws, L.sa);
         P2.n_problems = 1;
@@ -560,6 +561,7 @@ moe_status_t run_expert_ffn_pairs(const moe_config_t* c, const void* x, const in
         p.out = y;
         p.ld_out = c->H;
         p.row_w = g.w_perm;
+        p.out_f32 = c->k == 1;
         P2.n_problems = 1;
         if (Is > 0) {
             moe::PairProblem& q = P2.p[1];
@@ -667,6 +669,7 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
         p.out = y;
         p.ld_out = c->H;
         p.row_w = g.w_perm;
+        p.out_f32 = c->k == 1;
         P2.n_problems = 1;
         if (Is > 0) {
             moe::GemmProblem& q = P2.p[1];
@@ -714,7 +717,8 @@ moe_status_t run_combine(const moe_config_t* c, const void* y, const int32_t* po
                          const void* y_shared, void* out, cudaStream_t s,
                          const void* residual = nullptr) {
     moe::CombineArgs a;
-    a.y = static_cast<const uint16_t*>(y);
+    a.y = y;
+    a.y_f32 = c->k == 1;
     a.pos = pos;
     a.y_shared = static_cast<const float*>(y_shared);
     a.residual = static_cast<const uint16_t*>(residual);

@@ -239,7 +239,9 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
 }
 
 // out[t] = bf16( sum_j y[pos[t*k + j]] + y_shared[t] (+ residual[t]) ), 8 columns per
-// thread, one fp32 sum in that order and one rounding.
+// thread, one fp32 sum in that order and one rounding.  y is bf16, or fp32
+// when k = 1 (a single routed row per token: its rounding to bf16 would not be
+// averaged with other experts' and would be the largest error of the sum).
 __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
     const int t = blockIdx.x;
     const int c = blockIdx.y * blockDim.x + threadIdx.x;  // 16-byte chunk
@@ -250,7 +252,16 @@ __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
     for (int j = 0; j < a.k; ++j) {
         const int r = a.pos[(size_t)t * a.k + j];
         if (r < 0) continue;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.y + (size_t)r * a.H) + c);
+        if (a.y_f32) {
+            const float4* yr = reinterpret_cast<const float4*>(
+                                   static_cast<const float*>(a.y) + (size_t)r * a.H) + 2 * c;
+            const float4 v0 = __ldg(yr), v1 = __ldg(yr + 1);
+            acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+            acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+            continue;
+        }
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+                                  static_cast<const uint16_t*>(a.y) + (size_t)r * a.H) + c);
         const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -49,12 +49,13 @@ struct GatherArgs {
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
 
 struct CombineArgs {
-    const uint16_t* y;        // bf16 [T*k, H]
+    const void* y;            // [T*k, H]: bf16, or fp32 with y_f32
     const int32_t* pos;       // [T*k]
     const float* y_shared;    // fp32 [T, H] or null
     const uint16_t* residual; // bf16 [T, H] added in the same fp32 sum, or null
     uint16_t* out;            // bf16 [T, H]
     int T, k, H;
+    int y_f32;                // routed outputs stored fp32 (k = 1)
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 

@@ -109,8 +109,73 @@ def test_layer_small_shapes_against_oracle(B, W, case):
     print("%s: rel-L2 %.2e, max-abs/rms %.2e, near-ties %d" % (name, rel, mx, ties))
 
 
-def test_stage_entry_points_match_forward(B, W):
-    wl = W.Workload("stages", T=200, H=1024, E=64, k=6, I=256, n_shared=1, seed=5)
+# routing options and the largest configurations the router accepts
+ROUTING_EDGE = [
+    # name, T, H, E, k, I, n_shared, n_group, topk_group, norm_topk_prob, routed_scaling_factor
+    ("no_norm_rsf2.5", 200, 512, 64, 3, 128, 1, 1, 1, False, 2.5),
+    ("norm_rsf0.5", 200, 512, 64, 6, 128, 1, 1, 1, True, 0.5),
+    ("k1_norm", 150, 512, 32, 1, 128, 1, 1, 1, True, 1.0),
+    ("max_E_k", 96, 128, 1024, 32, 128, 1, 1, 1, True, 1.0),
+    ("max_groups", 96, 128, 1024, 16, 128, 0, 32, 4, True, 1.0),
+    ("E768_groups", 130, 256, 768, 8, 128, 1, 8, 3, True, 1.0),
+]
+
+
+@pytest.mark.parametrize("case", ROUTING_EDGE, ids=[c[0] for c in ROUTING_EDGE])
+def test_routing_options_and_max_sizes_against_oracle(B, W, case):
+    name, T, H, E, k, I, S, G, tg, norm, rsf = case
+    wl = W.Workload(name, T=T, H=H, E=E, k=k, I=I, n_shared=S, n_group=G, topk_group=tg,
+                    norm_topk_prob=norm, routed_scaling_factor=rsf,
+                    seed=sum(name.encode()) % 1000)
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl)
+    out, ws = run_forward(B, cfg, inp)
+    L, idx, w, ties = check_routing(B, cfg, ws, inp)
+    check_permutation(B, cfg, ws, idx)
+    if k == 1 and norm:
+        assert (w == np.float32(rsf)).all()
+    ref = oracle_layer_on_tokens(cfg, inp, idx, w, np.arange(T))
+    rel, mx = assert_close_bf16(out.float().cpu().numpy(), ref, name)
+    print("%s: rel-L2 %.2e, max-abs/rms %.2e, near-ties %d" % (name, rel, mx, ties))
+
+
+def test_one_expert_takes_every_token(B, W):
+    """A bias that makes one expert every token's first choice: its segment
+    holds all T rows, a dozen CTA-pair token tiles of one expert."""
+    wl = W.Workload("hot", T=3000, H=640, E=32, k=2, I=384, n_shared=1, seed=11)
+    inp = W.make_inputs(wl, device="cuda")
+    inp["bias"] = torch.zeros(32, device="cuda")
+    inp["bias"][5] = 10.0
+    cfg = mk_cfg(B, wl)
+    out, ws = run_forward(B, cfg, inp)
+    L, idx, w, _ = check_routing(B, cfg, ws, inp)
+    offs = check_permutation(B, cfg, ws, idx)
+    assert (idx[:, 0] == 5).all() and offs[6] - offs[5] == wl.T
+    toks = np.unique(np.concatenate([np.random.default_rng(1).choice(wl.T, 48, replace=False),
+                                     [0, wl.T - 1]]))
+    ref = oracle_layer_on_tokens(cfg, inp, idx, w, toks)
+    assert_close_bf16(out[torch.as_tensor(toks, device="cuda")].float().cpu().numpy(), ref, "hot")
+
+
+def test_empty_batch_is_a_no_op(B, W):
+    """T = 0: every call validates its arguments and returns without a launch."""
+    wl = W.Workload("empty", T=4, H=512, E=32, k=4, I=128, seed=2)
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl, T=0)
+    ws = B.alloc_workspace(cfg)
+    out = torch.full((4, wl.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    B.moe_forward(cfg, inp["x"], inp["w_router"], inp["bias"], inp["w13"], inp["w2"],
+                  inp["w13s"], inp["w2s"], out, ws)
+    torch.cuda.synchronize()
+    B.moe_check_device_status(ws)
+    assert (out.float() == 7.0).all()
+
+
+@pytest.mark.parametrize("k", [6, 1])
+def test_stage_entry_points_match_forward(B, W, k):
+    """The step calls reproduce moe_forward bit for bit (with k = 1 the routed
+    outputs y are fp32)."""
+    wl = W.Workload("stages", T=200, H=1024, E=64, k=k, I=256, n_shared=1, seed=5)
     inp = W.make_inputs(wl, device="cuda")
     cfg = mk_cfg(B, wl)
     out, ws = run_forward(B, cfg, inp)
@@ -128,7 +193,7 @@ def test_stage_entry_points_match_forward(B, W):
     rows = torch.empty((T * k,), dtype=torch.int32, device=dev)
     pos = torch.empty((T * k,), dtype=torch.int32, device=dev)
     B.moe_permute(cfg, idx, offsets, rows, pos, ws2)
-    y = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T * k, H), dtype=torch.float32 if k == 1 else torch.bfloat16, device=dev)
     ysh = torch.empty((T, H), dtype=torch.float32, device=dev)
     B.moe_expert_ffn(cfg, inp["x"], offsets, rows, pos, w, inp["w13"], inp["w2"], inp["w13s"],
                      inp["w2s"], y, ysh, ws2)
