@@ -273,6 +273,27 @@ def layer_work(wl, touched: int):
     return {"flops": flops, "bytes": bytes_, "g1_flops": g1_flops, "g1_bytes": g1_bytes}
 
 
+def layer_config(wl, args, world):
+    """The workload's identity, the same in both arms' JSON lines."""
+    el = 1 if wl.dtype == "fp8" else 2
+    sc = 4.0 / (128 * 128) if wl.dtype == "fp8" else 0.0
+    resident = (wl.E * 3 * wl.H * wl.I + 3 * wl.H * wl.Is) * (el + sc)
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+            "n_shared": wl.n_shared, "n_group": wl.n_group, "topk_group": wl.topk_group,
+            "block": "h + MoE(RMSNorm(h))" if args.block else None,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2: %.1f GB of expert weights resident, each step streams "
+                  "those of the experts it touches" % (resident / 1e9)}
+
+
+def dsa_config(wl, args):
+    return {"workload": wl.name, "Sq": wl.Sq, "Sk": wl.Sk, "n_heads": wl.n_heads,
+            "head_dim": 128, "topk": wl.topk, "causal": wl.causal,
+            "sorted": not args.dsa_unsorted, "q_offset": wl.q_offset,
+            "l2": "inputs larger than L2: %.0f MB of keys and %.0f MB of scores per step"
+                  % (wl.Sk * wl.n_heads * 256 / 1e6, wl.Sq * wl.Sk * 4 / 1e6)}
+
+
 # ---------------------------------------------------------------- our arm
 
 def workload_of(args):
@@ -545,15 +566,16 @@ def run_reference(args, world, rank):
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": wl.Sq / value * 1e3, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl.name, "Sq": wl.Sq, "Sk": wl.Sk, "n_heads": wl.n_heads,
-                           "topk": wl.topk},
+                "config": dsa_config(wl, args),
                 "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads,
                                  "kind": "oracle", "sample": sample},
                 "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
-    wl = W.WORKLOADS[args.workload]
+    wl = workload_of(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.make_inputs(wl, device=dev)
+    if args.block:  # the pre-norm block: the oracle's RMSNorm, layer and residual add
+        inp["gamma"] = W.make_norm_weight(wl, device=dev, seed=wl.seed)
     per_step = max(2.0, args.cpu_seconds / max(1, args.steps + args.warmup))
     rates = []
     for i in range(args.warmup + args.steps):
@@ -566,8 +588,7 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
-                       "I": wl.I, "n_shared": wl.n_shared},
+            "config": layer_config(wl, args, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -731,12 +752,7 @@ def dsa_main(args, world, rank, local):
     line = {"metric": DSA_METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": r["ms"] / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "Sq": wl.Sq, "Sk": wl.Sk, "n_heads": wl.n_heads,
-                       "head_dim": 128, "topk": wl.topk, "causal": wl.causal,
-                       "sorted": not args.dsa_unsorted,
-                       "q_offset": wl.q_offset,
-                       "l2": "inputs larger than L2: %.0f MB of keys and %.0f MB of scores per step"
-                             % (wl.Sk * wl.n_heads * 256 / 1e6, wl.Sq * wl.Sk * 4 / 1e6)},
+            "config": dsa_config(wl, args),
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
                          "frac": ach / pk, "traffic": profile_traffic("dsa_scores", None, wl.name),
                          "peak_kind": "bf16 sustained",
@@ -828,13 +844,9 @@ def main():
             "warmup": args.warmup, "ms_per_step": layer_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
-                       "I": wl.I, "n_shared": wl.n_shared, "n_group": wl.n_group,
-                       "topk_group": wl.topk_group, "experts_touched": r["touched"],
-                       "block": "h + MoE(RMSNorm(h))" if args.block else None,
-                       "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
-                             % (work["bytes"] / 1e9)},
+            "config": layer_config(wl, args, world),
+            "routing": {"experts_touched": r["touched"],
+                        "algorithmic_gb_per_step": work["bytes"] / 1e9},
             "roofline": roof, "layer_roofline": layer,
             "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
             "gpu_launches": r["launches"], "clocks": r["clocks"],
