@@ -62,3 +62,12 @@ def test_reference_arm_under_torchrun_two_ranks():
     line = lines[0]
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+    # the contract's keys, and the same workload identity our arm prints
+    for key in ("metric", "unit", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "e2e"):
+        assert key in line, key
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    import argparse
+    import bench
+    args = argparse.Namespace(workload="tiny", T=None, E=None, block=False)
+    assert line["config"] == bench.layer_config(bench.workload_of(args), args, 2)
