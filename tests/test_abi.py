@@ -53,6 +53,12 @@ def test_workspace_size_and_offsets(B):
     assert len(set(offs)) == len(offs)
     big = cfg(B, T=8192)
     assert B.workspace_size(big) > n
+    # the routed outputs y hold fp32 rows when k = 1, bf16 otherwise: the next
+    # region starts at least T*k*H*4 (resp. *2) bytes after y
+    for kk, el in ((1, 4), (2, 2)):
+        c1 = cfg(B, k=kk)
+        y0, ysh0 = B.workspace_offset(c1, "y"), B.workspace_offset(c1, "y_shared")
+        assert ysh0 - y0 >= T * kk * H * el
 
 
 @pytest.mark.parametrize("kw", [dict(H=100), dict(E=33), dict(E=0), dict(k=0), dict(k=300),
