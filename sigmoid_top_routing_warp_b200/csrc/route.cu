@@ -79,8 +79,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(const RouteArgs a) {
 #pragma unroll
     for (int i = 0; i < VPL; ++i) lg[i] = __ldg(row + i);
     if (a.n_split > 1) {
-        // K-slice partials of the router GEMM, summed in slice order (the
-        // loads of all slices are issued before the adds)
+        // K-slice partials of the router GEMM, summed in slice order
         for (int sp = 1; sp < a.n_split; ++sp) {
             float part[VPL];
 #pragma unroll
