@@ -57,6 +57,8 @@ def parse():
                     help="DSA workloads: indices by key order (no sort by score)")
     ap.add_argument("--block", action="store_true",
                     help="time the pre-norm block out = h + MoE(RMSNorm(h)) (moe_forward_block)")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="default decode run: skip the prefill object (T=8192 Zipf) in the line")
     return ap.parse_args()
 
 
@@ -119,7 +121,7 @@ def dist_teardown(world):
 
 class ClockSampler:
     """SM clock and throttle reasons sampled during the timed region: an NVML
-    polling thread (every 2 ms), or nvidia-smi at 50 ms where NVML is absent."""
+    polling thread (every 0.5 ms), or nvidia-smi at 50 ms where NVML is absent."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -156,7 +158,7 @@ class ClockSampler:
                                              int(get_reasons(h))))
                     except Exception:
                         pass
-                    time.sleep(0.002)
+                    time.sleep(0.0005)
 
             import threading
             self.thread = threading.Thread(target=poll, daemon=True)
@@ -394,6 +396,7 @@ def run_ours(args, world, rank, local):
     stage_ms = stages.mean(0)
 
     graph_ms = None
+    graph_clocks = None
     if not args.eager:
         # one step captured on a side stream, replayed K times on it
         gs = torch.cuda.Stream(dev)
@@ -408,21 +411,23 @@ def run_ours(args, world, rank, local):
         barrier(world)
         g0 = torch.cuda.Event(enable_timing=True)
         g1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(gs):
-            g0.record(gs)
-            for _ in range(K):
-                graph.replay()
-            g1.record(gs)
-        torch.cuda.synchronize(dev)
+        with ClockSampler(dev.index) as gclk:
+            with torch.cuda.stream(gs):
+                g0.record(gs)
+                for _ in range(K):
+                    graph.replay()
+                g1.record(gs)
+            torch.cuda.synchronize(dev)
         barrier(world)
         graph_ms = max_over_ranks(world, g0.elapsed_time(g1))
+        graph_clocks = gclk.summary()
         B.moe_check_device_status(ws)
         del graph
     if args.no_e2e:
         return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
                 "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": None,
                 "launches": launches_per_step(B, cfg, args.block) * K, "B": B,
-                "graph_ms": graph_ms}
+                "graph_ms": graph_ms, "graph_clocks": graph_clocks, "ws": ws}
     # end to end through the C ABI with host buffers, as a serving loop runs it:
     # every step copies its x from pinned host memory and its out back, on copy
     # streams with two device buffers each, so that step i's copies overlap the
@@ -474,7 +479,7 @@ def run_ours(args, world, rank, local):
     return {"wl": wl, "cfg": cfg, "inp": inp, "touched": touched, "ms": ms_max,
             "stage_ms": stage_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "launches": launches_per_step(B, cfg, args.block) * K, "B": B,
-            "graph_ms": graph_ms}
+            "graph_ms": graph_ms, "graph_clocks": graph_clocks, "ws": ws}
 
 
 # ---------------------------------------------------------------- oracle (CPU)
@@ -756,7 +761,10 @@ def dsa_main(args, world, rank, local):
     work = dsa_work(wl)
     value = world * wl.Sq * K / (r["ms"] / 1e3)
     ach = work["flops"] / (r["sc_ms"] / 1e3) / 1e12
-    pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # a K-step run of about a millisecond per step is a burst: the burst peak
+    # is the denominator, the sustained one beside it
+    pk = peaks["bf16_tflops"]
+    pk_sus = peaks.get("bf16_tflops_sustained", pk)
     tk_gbs = work["topk_bytes"] / (r["tk_ms"] / 1e3) / 1e9
     line = {"metric": DSA_METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": r["ms"] / K, "higher_is_better": True,
@@ -764,8 +772,8 @@ def dsa_main(args, world, rank, local):
             "config": dsa_config(wl, args),
             "roofline": {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
                          "frac": ach / pk, "traffic": profile_traffic("dsa_scores", None, wl.name),
-                         "peak_kind": "bf16 sustained",
-                         "frac_of_burst_peak": ach / peaks["bf16_tflops"],
+                         "peak_kind": "bf16 burst",
+                         "frac_of_sustained_peak": ach / pk_sus,
                          "kernel": "dsa_scores_kernel (w x ReLU(q.k) over heads)",
                          "algorithmic_per_launch": work["flops"], "launch_ms": r["sc_ms"],
                          "peak_source": peak_src},
@@ -787,6 +795,100 @@ def dsa_main(args, world, rank, local):
     dist_teardown(world)
 
 
+def routing_check(r):
+    """Near-tie count of the timed batch, with the oracle as the checker (part
+    of the CPU-baseline leg, outside the timed region): the oracle routes the
+    GPU's own fp32 logits; the indices and weights must equal the GPU's bit for
+    bit, and tokens whose k-th and (k+1)-th biased scores lie closer than 1e-4
+    are counted."""
+    from oracle import oracle as O
+    wl, B, cfg, ws = r["wl"], r["B"], r["cfg"], r["ws"]
+    L = B.ws_view(ws, cfg, "logits").cpu().numpy()
+    idx = B.ws_view(ws, cfg, "topk_idx").cpu().numpy()
+    w = B.ws_view(ws, cfg, "topk_w").cpu().numpy()
+    oc = O.Config(T=wl.T, H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=wl.n_shared,
+                  n_group=wl.n_group, topk_group=wl.topk_group, group_topn=wl.group_topn,
+                  norm_topk_prob=wl.norm_topk_prob,
+                  routed_scaling_factor=wl.routed_scaling_factor)
+    oidx, ow, gap = O.route(oc, L, r["inp"]["bias"].cpu().numpy())
+    exact = bool((idx == oidx).all() and (w.view(np.uint32) == ow.view(np.uint32)).all())
+    return {"near_ties": int((gap < 1e-4).sum()), "near_tie_gap": 1e-4, "tokens": wl.T,
+            "bit_exact_vs_oracle": exact}
+
+
+def layer_line(args, r, peaks, peak_src, world):
+    """The JSON line of one timed layer workload (our arm)."""
+    wl, K = r["wl"], args.steps
+    work = layer_work(wl, r["touched"])
+    step_ms_total = r["graph_ms"] if r["graph_ms"] is not None else r["ms"]
+    value = world * wl.T * K / (step_ms_total / 1e3)
+    stage_names = r["B"].STAGE_NAMES
+    g1_ms = float(r["stage_ms"][3])
+    pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
+    fp8 = wl.dtype == "fp8"
+    # token-major fp8 kernel: hidden and intermediate sizes multiples of 512
+    tm = fp8 and wl.H % 512 == 0 and wl.I % 512 == 0
+    kind = ("gate_up_fp8_tm" if tm else "gate_up_fp8" if fp8 else
+            "gate_up_prefill" if pair else "gate_up_decode")
+    traffic = profile_traffic(kind, work["g1_bytes"], wl.name + ("_block" if args.block else ""))
+    if fp8:  # no fp8 peak is measured: the bf16 peaks x the nominal fp8/bf16 ratio 2
+        peaks = dict(peaks)
+        for key in ("bf16_tflops", "bf16_tflops_sustained"):
+            if key in peaks:
+                peaks[key] = 2.0 * peaks[key]
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    pk_name = "fp8 (assumed 2x the measured bf16 peak; no fp8 peak measured)" if fp8 else "bf16"
+    hbm_bound = work["bytes"] / (peaks["hbm_gbs"] * 1e9) >= work["flops"] / (burst * 1e12)
+    if hbm_bound:
+        ach = work["g1_bytes"] / (g1_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic}
+    else:
+        # K steps of a few ms are a short burst, not a seconds-long loop: the
+        # burst tensor peak is the denominator; the sustained one is beside it
+        ach = work["g1_flops"] / (g1_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s",
+                "frac": ach / burst, "traffic": traffic,
+                "peak_kind": pk_name + " burst",
+                "frac_of_sustained_peak": ach / sustained}
+    kname = ("fp8_tm_gemm_kernel<SWIGLU>" if tm else "fp8_gemm_kernel<SWIGLU>" if fp8 else
+             "pair_gemm_kernel<SWIGLU>" if pair else "grouped_gemm_kernel<SWIGLU,16>")
+    roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
+                 "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
+                 "launch_ms": g1_ms, "peak_source": peak_src})
+    layer_ms = step_ms_total / K
+    layer = {"ms": layer_ms,
+             "hbm_gbs": work["bytes"] / (layer_ms / 1e3) / 1e9,
+             "tflops": work["flops"] / (layer_ms / 1e3) / 1e12,
+             "t_roof_ms": 1e3 * max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                                    work["flops"] / (burst * 1e12)),
+             "tensor_peak_tflops": burst, "tensor_peak_kind": pk_name + " burst"}
+    layer["frac_of_roofline"] = layer["t_roof_ms"] / layer_ms
+    if not hbm_bound:
+        layer["frac_of_sustained_roofline"] = 1e3 * max(
+            work["bytes"] / (peaks["hbm_gbs"] * 1e9), work["flops"] / (sustained * 1e12)) / layer_ms
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": layer_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+            "data": "synthetic",
+            "config": layer_config(wl, args, world),
+            "routing": {"experts_touched": r["touched"],
+                        "algorithmic_gb_per_step": work["bytes"] / 1e9},
+            "roofline": roof, "layer_roofline": layer,
+            "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
+            "gpu_launches": r["launches"],
+            # the clocks of the region `value` comes from (graph replay by default)
+            "clocks": r["graph_clocks"] if r["graph_clocks"] is not None else r["clocks"],
+            "clocks_eager": r["clocks"],
+            "graph": None if r["graph_ms"] is None else {
+                "ms_per_step": r["graph_ms"] / K, "eager_ms_per_step": r["ms"] / K},
+            "e2e": None if r["e2e_ms"] is None else {
+                "value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
+    return line
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
@@ -801,73 +903,32 @@ def main():
         return
     peaks, peak_src = load_peaks()
     r = run_ours(args, world, rank, local)
-    wl, K = r["wl"], args.steps
-    work = layer_work(wl, r["touched"])
-    step_ms_total = r["graph_ms"] if r["graph_ms"] is not None else r["ms"]
-    value = world * wl.T * K / (step_ms_total / 1e3)
-    stage_names = r["B"].STAGE_NAMES
-    g1_ms = float(r["stage_ms"][3])
-    pair = r["cfg"].T * r["cfg"].k / r["cfg"].E > 96.0 and wl.dtype != "fp8"
-    fp8 = wl.dtype == "fp8"
-    # token-major fp8 kernel: hidden and intermediate sizes multiples of 512
-    tm = fp8 and wl.H % 512 == 0 and wl.I % 512 == 0
-    kind = ("gate_up_fp8_tm" if tm else "gate_up_fp8" if fp8 else
-            "gate_up_prefill" if pair else "gate_up_decode")
-    traffic = profile_traffic(kind, work["g1_bytes"], wl.name + ("_block" if args.block else ""))
-    if fp8:  # the fp8 tensor peak: the measured bf16 peaks x the nominal fp8/bf16 ratio 2
-        peaks = dict(peaks)
-        for key in ("bf16_tflops", "bf16_tflops_sustained"):
-            if key in peaks:
-                peaks[key] = 2.0 * peaks[key]
-    hbm_bound = work["bytes"] / (peaks["hbm_gbs"] * 1e9) >= work["flops"] / (
-        peaks["bf16_tflops"] * 1e12)
-    if hbm_bound:
-        ach = work["g1_bytes"] / (g1_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": traffic}
-    else:
-        # the gate/up GEMM runs inside a multi-millisecond step, back to back:
-        # the sustained (power-capped) tensor peak is its denominator
-        ach = work["g1_flops"] / (g1_ms / 1e3) / 1e12
-        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
-                "frac": ach / pk, "traffic": traffic,
-                "peak_kind": "fp8 sustained (2x measured bf16)" if fp8 else "bf16 sustained",
-                "frac_of_burst_peak": ach / peaks["bf16_tflops"]}
-    kname = ("fp8_tm_gemm_kernel<SWIGLU>" if tm else "fp8_gemm_kernel<SWIGLU>" if fp8 else
-             "pair_gemm_kernel<SWIGLU>" if pair else "grouped_gemm_kernel<SWIGLU,16>")
-    roof.update({"kernel": kname + " (gate/up GEMM + SwiGLU)",
-                 "algorithmic_per_launch": work["g1_bytes"] if hbm_bound else work["g1_flops"],
-                 "launch_ms": g1_ms, "peak_source": peak_src})
-    layer_ms = step_ms_total / K
-    tensor_pk = peaks["bf16_tflops"] if hbm_bound else peaks.get("bf16_tflops_sustained",
-                                                                     peaks["bf16_tflops"])
-    layer = {"ms": layer_ms,
-             "hbm_gbs": work["bytes"] / (layer_ms / 1e3) / 1e9,
-             "tflops": work["flops"] / (layer_ms / 1e3) / 1e12,
-             "t_roof_ms": 1e3 * max(work["bytes"] / (peaks["hbm_gbs"] * 1e9),
-                                    work["flops"] / (tensor_pk * 1e12)),
-             "tensor_peak_tflops": tensor_pk}
-    layer["frac_of_roofline"] = layer["t_roof_ms"] / layer_ms
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": layer_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
-            "data": "synthetic",
-            "config": layer_config(wl, args, world),
-            "routing": {"experts_touched": r["touched"],
-                        "algorithmic_gb_per_step": work["bytes"] / 1e9},
-            "roofline": roof, "layer_roofline": layer,
-            "stages_ms": {n: float(v) for n, v in zip(stage_names, r["stage_ms"])},
-            "gpu_launches": r["launches"], "clocks": r["clocks"],
-            "graph": None if r["graph_ms"] is None else {
-                "ms_per_step": r["graph_ms"] / K, "eager_ms_per_step": r["ms"] / K},
-            "e2e": None if r["e2e_ms"] is None else {
-                "value": world * wl.T * K / (r["e2e_ms"] / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2}}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, sample = oracle_sample(wl, r["inp"], args.cpu_seconds)
+    line = layer_line(args, r, peaks, peak_src, world)
+    cpu_leg = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if cpu_leg:
+        line["routing"].update(routing_check(r))
+        v, threads, sample = oracle_sample(r["wl"], r["inp"], args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": sample}
+    # The default run also times the prefill workload (T = 8192, Zipf loads),
+    # the metric's tensor-bound configuration, with the same K and W; decode
+    # stays the headline value.
+    if (args.workload == "decode" and not args.no_prefill and not args.block
+            and args.T is None and args.E is None):
+        del r
+        torch.cuda.empty_cache()
+        pargs = argparse.Namespace(**{**vars(args), "workload": "prefill", "no_e2e": True})
+        rp = run_ours(pargs, world, rank, local)
+        pl = layer_line(pargs, rp, peaks, peak_src, world)
+        line["prefill"] = {
+            "workload": "prefill", "config": pl["config"], "value": pl["value"], "unit": UNIT,
+            "ms_per_step": pl["ms_per_step"], "tflops": pl["layer_roofline"]["tflops"],
+            "roofline": pl["roofline"], "layer_roofline": pl["layer_roofline"],
+            "stages_ms": pl["stages_ms"], "clocks": pl["clocks"],
+            "clocks_eager": pl["clocks_eager"], "graph": pl["graph"],
+            "gpu_launches": pl["gpu_launches"], "routing": pl["routing"]}
+        if cpu_leg:
+            line["prefill"]["routing"].update(routing_check(rp))
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist_teardown(world)

@@ -48,9 +48,9 @@ typedef struct {
 
 /* Bytes of workspace dsa_index_scores / dsa_indexer need: a 256-byte status
  * block, then (dsa_indexer) the fp32 score matrix [Sq, Sk].  0 if invalid.
- * The workspace must be zero-filled before its first use: the status block
- * holds the status word and the score kernel's tile-claim counters, which
- * every call leaves at zero. */
+ * The status block holds the status word (word 0, which must start at zero)
+ * and the score kernel's tile-claim counters, which every score launch
+ * zeroes on its stream first. */
 size_t dsa_workspace_size(const dsa_config_t* cfg);
 
 /* Scores.  q bf16 [Sq, n_heads, 128], k bf16 [Sk, n_heads, 128] (16-byte

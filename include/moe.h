@@ -122,9 +122,11 @@ const char* moe_get_last_error(void);
  * (0 if the configuration is invalid; see moe_get_last_error).  The
  * workspace holds logits, routing, the dispatch plan, the gathered
  * activations and the intermediate expert outputs; it must be 256-byte
- * aligned and zero-filled before its first use: its first 256 bytes hold the
- * status word and the GEMMs' tile-claim counters, which every call leaves at
- * zero (moe_check_device_status clears the status word). */
+ * aligned.  Its first 256 bytes hold the status word (word 0) and the
+ * persistent GEMMs' tile-claim counters (words 16..63).  Every call that
+ * launches a GEMM zeroes the counter words on its stream first, so the
+ * workspace needs no zero-fill; the status word must start at zero (a
+ * zero-filled buffer, or moe_check_device_status after an error). */
 size_t moe_workspace_size(const moe_config_t* cfg);
 
 /* Router: steps a1-a4.  Page: mlqm.cn 稀疏激活 (sigmoid, noaux_tc,
@@ -170,7 +172,11 @@ moe_status_t moe_permute(const moe_config_t* cfg, const int32_t* topk_idx, int32
  *     MOE_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (a one-time set-up per device); make that first
- *     call before any stream capture.
+ *     call before any stream capture.  The address belongs to the device's
+ *     CUDA context: when that context is replaced (cudaDeviceReset), the next
+ *     call sees a new context id and looks the address up again, so that call
+ *     too should come before any capture.
+ *   - T = 0 writes offsets[0..E] = 0, as moe_permute does.
  *   - Every call shares the one array: calls that overlap on the GPU race on
  *     it and must not be issued.
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
@@ -278,8 +284,53 @@ moe_status_t moe_forward_block(const moe_config_t* cfg, const void* h, const voi
  * input of moe_forward_block).  Returns (size_t)-1 if invalid. */
 size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
 
-/* Synchronise `stream`, read and clear the device status word in `ws`.
- * Returns MOE_OK, or MOE_ERR_TIMEOUT if a kernel gave up a bounded wait.  */
+/* ------------------------------------------------------------------------
+ * Backward pass (training side of the layer), bf16 layers.  The pages give
+ * the forward pass only (Deep Dive §3.1 gate -> scores -> top-k ->
+ * renormalise -> shared + weighted routed sum, §8.2 gmm1 -> swiglu -> gmm2;
+ * mlqm.cn 稀疏激活: sigmoid scores, noaux_tc, norm_topk_prob); this is the
+ * chain rule through it with the expert choice held fixed, for the loss
+ * sum(out * dout).  The choice (top-k of score + bias) is piecewise constant:
+ * no gradient flows through it and the expert bias gets none.
+ *
+ * Bytes of workspace moe_backward needs (256-byte aligned; no zero-fill
+ * needed): the dispatch plan, rows padded per expert to multiples of 16, the
+ * recomputed gate/up pre-activations and the intermediate gradients.  0 if
+ * the configuration is invalid.                                             */
+size_t moe_backward_workspace_size(const moe_config_t* cfg);
+
+/*   x         bf16 [T, H]        the forward's input
+ *   w_router  bf16 [E, H]
+ *   logits    fp32 [T, E]        the forward's router logits (moe_route)
+ *   topk_idx  int32 [T, k]       the forward's choice
+ *   topk_w    fp32 [T, k]        the forward's routing weights
+ *   w13, w2, w13s, w2s           the weights, as for moe_forward
+ *   dout      bf16 [T, H]        gradient of the loss at the layer output
+ *   dx        bf16 [T, H]  out   gradient at x (routed + shared + router),
+ *                                an fp32 sum rounded once
+ *   dw_router fp32 [E, H]  out
+ *   dw13      fp32 [E, 2I, H] out, dw2 fp32 [E, H, I] out (zero for an
+ *                                expert no token chose)
+ *   dw13s     fp32 [2 Is, H] out, dw2s fp32 [H, Is] out (n_shared > 0)
+ *   dlogits   fp32 [T, E]  out   gradient at the router logits, zero off the
+ *                                chosen experts; may be NULL
+ *   ws        moe_backward_workspace_size bytes
+ * All outputs are overwritten.  Pointers to bf16 data and every output
+ * except dlogits must be 16-byte aligned.  fp8 layers return
+ * MOE_ERR_UNSUPPORTED.                                                      */
+moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_router,
+                          const float* logits, const int32_t* topk_idx, const float* topk_w,
+                          const void* w13, const void* w2, const void* w13s, const void* w2s,
+                          const void* dout, void* dx, float* dw_router, float* dw13, float* dw2,
+                          float* dw13s, float* dw2s, float* dlogits, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Synchronise `stream`, read the workspace status block of `ws` (the layer's
+ * or the DSA indexer's) and clear it.  Returns MOE_OK; MOE_ERR_TIMEOUT if a
+ * kernel gave up a bounded wait; or MOE_ERR_WORKSPACE if a tile-claim counter
+ * was non-zero after the stream drained, i.e. a claiming launch stopped
+ * part-way (its output is incomplete).  Either way the block is zero after
+ * the call, so the next call on the workspace starts clean.               */
 moe_status_t moe_check_device_status(void* ws, moe_stream_t stream);
 
 #ifdef __cplusplus

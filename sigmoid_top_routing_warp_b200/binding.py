@@ -35,6 +35,7 @@ EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", 
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
             "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
             "moe_quantize_act", "moe_rmsnorm", "moe_forward_block",
+            "moe_backward_workspace_size", "moe_backward",
             "dsa_workspace_size", "dsa_workspace_scores_offset", "dsa_index_scores",
             "dsa_index_topk", "dsa_indexer")
 
@@ -129,6 +130,10 @@ _lib.moe_permute_noalloc.restype = ctypes.c_int
 _lib.moe_permute_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P]
 _lib.moe_quantize_act.restype = ctypes.c_int
 _lib.moe_quantize_act.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
+_lib.moe_backward_workspace_size.restype = ctypes.c_size_t
+_lib.moe_backward_workspace_size.argtypes = [_CFG]
+_lib.moe_backward.restype = ctypes.c_int
+_lib.moe_backward.argtypes = [_CFG] + [_P] * 18 + [ctypes.c_size_t, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -268,6 +273,30 @@ def moe_quantize_act(x, q, scale, stream=None):
     rows, cols = x.shape
     _check(_lib.moe_quantize_act(_ptr(x), rows, cols, _ptr(q), _ptr(scale), _stream(stream)),
            "moe_quantize_act")
+
+
+def backward_workspace_size(cfg: MoeConfig) -> int:
+    c = cfg.c()
+    n = _lib.moe_backward_workspace_size(ctypes.byref(c))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_backward_workspace_size")
+    return n
+
+
+def alloc_backward_workspace(cfg: MoeConfig, device="cuda") -> torch.Tensor:
+    """A workspace of moe_backward_workspace_size bytes (256-byte aligned)."""
+    return torch.zeros(backward_workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def moe_backward(cfg, x, w_router, logits, topk_idx, topk_w, w13, w2, w13s, w2s, dout, dx,
+                 dw_router, dw13, dw2, dw13s, dw2s, ws, dlogits=None, stream=None):
+    """Gradients of sum(out * dout) with the forward's choice held fixed."""
+    c = cfg.c()
+    _check(_lib.moe_backward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(logits),
+                             _ptr(topk_idx), _ptr(topk_w), _ptr(w13), _ptr(w2), _ptr(w13s),
+                             _ptr(w2s), _ptr(dout), _ptr(dx), _ptr(dw_router), _ptr(dw13),
+                             _ptr(dw2), _ptr(dw13s), _ptr(dw2s), _ptr(dlogits), _ptr(ws),
+                             ws.numel(), _stream(stream)), "moe_backward")
 
 
 def moe_check_device_status(ws, stream=None):

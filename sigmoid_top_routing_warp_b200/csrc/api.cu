@@ -243,6 +243,11 @@ moe_status_t sm_count(int* n) {
     return MOE_OK;
 }
 
+moe_status_t reset_claims(void* ws, cudaStream_t s) {
+    MOE_CUDA(moe::reset_claim_counters(static_cast<int*>(ws), s), "claim-counter reset");
+    return MOE_OK;
+}
+
 #define MOE_TRY(x)                          \
     do {                                    \
         moe_status_t st_ = (x);             \
@@ -795,6 +800,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const void* w_rou
     MOE_TRY(need(topk_w, "topk_w"));
     if (cfg->T == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MOE_TRY(reset_claims(ws, s));
     const Layout L = layout(cfg);
     const int split = router_split(cfg);
     float* gemm_out = split > 1 ? at<float>(ws, L.rpart) : logits;
@@ -852,6 +858,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_
         MOE_TRY(need16(y_shared, "y_shared"));
     }
     if (cfg->T == 0) return MOE_OK;
+    MOE_TRY(reset_claims(ws, static_cast<cudaStream_t>(stream)));
     Weights W{w13, w2, w13s, w2s, w13_scale, w2_scale, w13s_scale, w2s_scale};
     return run_expert_ffn(cfg, x, offsets, pos, topk_w, W, y, y_shared, ws,
                           static_cast<cudaStream_t>(stream), nullptr, nullptr);
@@ -917,6 +924,7 @@ moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* ga
     const int split = router_split(cfg);
     float* gemm_out = split > 1 ? at<float>(ws, L.rpart) : logits;
     MOE_TRY(mark(0));
+    MOE_TRY(reset_claims(ws, s));
     const void* xin = x;
     if (gamma) {
         void* u = at<void>(ws, L.u);
@@ -1008,12 +1016,23 @@ moe_status_t moe_check_device_status(void* ws, moe_stream_t stream) {
     if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
-    int word = 0;
-    MOE_CUDA(cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost), "status read");
-    const int zero = 0;
-    MOE_CUDA(cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice), "status clear");
-    if (word & moe::DEV_STATUS_TIMEOUT)
-        return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", word);
+    int words[moe::kStatusWords];
+    MOE_CUDA(cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost), "status read");
+    int dirty = -1;
+    for (int i = moe::kSchedFirstWord; i < moe::kStatusWords; ++i)
+        if (words[i] != 0) {
+            dirty = i;
+            break;
+        }
+    const int zero[moe::kStatusWords] = {};
+    MOE_CUDA(cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
+    if (words[0] & moe::DEV_STATUS_TIMEOUT)
+        return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", words[0]);
+    if (dirty >= 0)
+        return fail(MOE_ERR_WORKSPACE,
+                    "tile-claim counter word %d was %d after the stream drained: a launch "
+                    "stopped part-way (the counters are now cleared)",
+                    dirty, words[dirty]);
     return MOE_OK;
 }
 
@@ -1026,6 +1045,23 @@ moe_status_t api_check_config(const moe_config_t* c) { return check_config(c); }
 moe_status_t api_fail(moe_status_t st, const char* msg) { return fail(st, "%s", msg); }
 void api_clear_error() { g_err[0] = 0; }
 moe_status_t api_sm_count(int* n) { return sm_count(n); }
+
+// bf16 row-major [rows, cols] as a 2-D tensor, box {box_cols, box_rows}, 128-byte swizzle.
+moe_status_t api_make_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                                  uint32_t box_cols, uint32_t box_rows, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
 
 // bf16 3-D tensor map {d0, d1, d2} (d0 contiguous; byte strides of d1 and d2),
 // box {b0, b1, b2}, 128-byte swizzle.

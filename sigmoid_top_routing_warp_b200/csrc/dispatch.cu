@@ -300,4 +300,11 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Zero the tile-claim words of a workspace status block, in stream order
+// before a claiming launch (a memset node when captured in a graph).
+cudaError_t reset_claim_counters(int* status, cudaStream_t s) {
+    return cudaMemsetAsync(status + kSchedFirstWord, 0,
+                           (kStatusWords - kSchedFirstWord) * sizeof(int), s);
+}
+
 }  // namespace moe

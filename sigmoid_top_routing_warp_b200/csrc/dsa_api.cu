@@ -89,7 +89,9 @@ moe_status_t run_scores(const dsa_config_t* c, const void* q, const void* k, con
     a.status = static_cast<int*>(ws);
     int sms = 0;
     DSA_TRY(moe::api_sm_count(&sms));
-    cudaError_t e = moe::launch_dsa_scores(a, sms, s);
+    cudaError_t e = moe::reset_claim_counters(a.status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "claim-counter reset");
+    e = moe::launch_dsa_scores(a, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "DSA score kernel launch");
     return MOE_OK;
 }

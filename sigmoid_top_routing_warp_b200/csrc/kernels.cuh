@@ -10,6 +10,17 @@ namespace moe {
 // Device status word bits (stored in the workspace).
 enum : int { DEV_STATUS_TIMEOUT = 1 };
 
+// The workspace's first 256 bytes: word 0 is the status word; words
+// kSchedFirstWord .. kStatusWords - 1 hold the persistent GEMMs' tile-claim
+// counters (a claim counter and a finished-CTA count per kernel and
+// epilogue kind).  Every entry point that launches a claiming kernel zeroes
+// those words on its stream first, and the last CTA of each launch zeroes
+// its own pair again; a non-zero word after the stream has drained means a
+// launch stopped part-way.
+constexpr int kStatusWords = 64;
+constexpr int kSchedFirstWord = 16;
+cudaError_t reset_claim_counters(int* status, cudaStream_t s);
+
 // ---------------------------------------------------------------- router
 struct RouteArgs {
     const float* logits;  // [n_split, T, E]: logits, or K-slice partials summed in order
@@ -186,5 +197,53 @@ cudaError_t launch_fp8_gemm(int epi, int bn, const GemmParams& params, int grid,
 // multiple of 512, n_feat a multiple of 128, and the tsx / tsw maps.
 constexpr int kFp8TokTile = 128;
 cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cudaStream_t s);
+
+// ---------------------------------------------------------------- backward GEMMs
+// One problem of a backward grouped GEMM launch (gemm_bwd.cu).  The tensor-
+// memory accumulator of a tile is D[m, n] = sum_k A(m, k) B(n, k) over a
+// 128 x 128 tile, lane = m, column = n; each operand is K-major (a 2-D map
+// [rows, K], box {64, 128}) or MN-major (a 2-D map [K, MN], box {64, 64},
+// two boxes per stage).
+//   rows_as_k = 0: the N dimension runs over token rows, grouped by `seg`
+//     (per group: tiles of 128 rows, prefix `tstart`), K = [0, K); A's row
+//     coordinate is offset by group * a_grp_rows (the group's weights).
+//     Output out[row * ld_out + m].
+//   rows_as_k = 1: K runs over the token rows of a group, [seg[g], seg[g+1])
+//     (or [0, n_rows) without seg); tiles cover M x N per group.  Output
+//     out[g * out_grp + n * ld_out + m] (a group's weight gradient).
+enum BwdEpilogue : int { BEPI_STORE = 0, BEPI_DSWIGLU = 1 };
+struct BwdProblem {
+    CUtensorMap ta, tb;
+    int a_mn, b_mn;
+    int rows_as_k;
+    const int32_t* seg;       // [n_grp + 1] group row offsets, or null: one group [0, n_rows)
+    const int32_t* tstart;    // rows_as_k = 0 with seg: [n_grp + 1] prefix of 128-row tiles
+    int n_grp, n_rows;
+    int M, N, K;
+    int a_grp_rows;
+    void* out;
+    int ld_out;
+    long long out_grp;
+    int out_f32;
+    // BEPI_DSWIGLU (rows_as_k = 0, M = half): D[i, r] = dL/da'_r[i] before the
+    // routing weight; gu [rows, 2 half] (fp32) holds the gate (cols < half) and
+    // up pre-activations of each row
+    const float* gu;
+    int ld_gu, half;
+    const float* row_w;       // routing weight per row, or null (1)
+    uint16_t* dgu;            // [rows, ld_dgu]: dgate | dup (bf16)
+    int ld_dgu;
+    uint16_t* aw;             // [rows, ld_aw]: w * SiLU(g) * u (bf16)
+    int ld_aw;
+    float* dw_part;           // [rows, ld_dw]: sum over 32 features of a' * da, or null
+    int ld_dw;
+};
+constexpr int kBwdMaxProblems = 5;
+struct BwdParams {
+    BwdProblem p[kBwdMaxProblems];
+    int n_problems;
+    int* status;
+};
+cudaError_t launch_bwd_gemm(int epi, const BwdParams& params, int grid, cudaStream_t s);
 
 }  // namespace moe

@@ -19,11 +19,16 @@
 // device array, not a device address.  The device address is looked up once
 // per device with cudaGetSymbolAddress, with that device current, the first
 // time the entry point runs on that device; that first call should therefore
-// come before any stream capture.  Nothing here calls cudaMalloc, cudaFree or
-// any allocating library routine.
+// come before any stream capture.  The address belongs to the device's
+// current CUDA context: if that context is replaced (after cudaDeviceReset,
+// for example) the module may load elsewhere, so every call compares the
+// current context's id with the one recorded at set-up and repeats the
+// look-up when they differ.  Nothing here calls cudaMalloc, cudaFree or any
+// allocating library routine.
 #include "moe.h"
 #include "kernels.cuh"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -43,9 +48,37 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 int32_t* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context id of the look-up
 
-// Device address of the scratch array on the current device (set-up once
-// per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current CUDA context (0 if there is none yet).
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_ctx = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_ctx = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+        looked_up = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the scratch array on the current device: looked up once
+// per device, and again only if the device's context has changed since.
 moe_status_t scratch_on_current_device(int32_t** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -53,7 +86,8 @@ moe_status_t scratch_on_current_device(int32_t** out) {
     if (dev < 0 || dev >= kMaxDevices)
         return moe::api_fail(MOE_ERR_UNSUPPORTED, "device ordinal beyond the supported range");
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) {
@@ -63,6 +97,8 @@ moe_status_t scratch_on_current_device(int32_t** out) {
             return moe::api_fail(MOE_ERR_CUDA, msg);
         }
         g_scratch_addr[dev] = static_cast<int32_t*>(p);
+        // the look-up made the device's primary context current if none was
+        g_scratch_ctx[dev] = current_context_id();
     }
     *out = g_scratch_addr[dev];
     return MOE_OK;
@@ -88,7 +124,8 @@ extern "C" moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const int32
                  n, cfg->E, need, kNoAllocScratchInts);
         return moe::api_fail(MOE_ERR_UNSUPPORTED, msg);
     }
-    if (cfg->T == 0) return MOE_OK;
+    // T = 0 still launches: the single-block path writes offsets[0..E] = 0
+    // (as moe_permute does) and reads no scratch
     int32_t* scratch = nullptr;
     st = scratch_on_current_device(&scratch);
     if (st != MOE_OK) return st;

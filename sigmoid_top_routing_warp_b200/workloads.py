@@ -282,3 +282,10 @@ def make_dsa_inputs(wl: DsaWorkload, device="cpu", seed: int | None = None):
     return {"q": _normal_bf16((wl.Sq, wl.n_heads, D), 1.0, g, device),
             "k": _normal_bf16((wl.Sk, wl.n_heads, D), 1.0, g, device),
             "w": _normal_bf16((wl.Sq, wl.n_heads), wl.n_heads ** -0.5, g, device)}
+
+
+def make_grad_output(wl: Workload, device="cpu", seed: int | None = None) -> torch.Tensor:
+    """The upstream gradient of a backward step: dout [T, H] ~ N(0, 1) in bf16
+    (its own seed stream, so it never aliases the forward's draws)."""
+    seed = (wl.seed if seed is None else seed) + 7919
+    return _normal_bf16((wl.T, wl.H), 1.0, _gen(torch.device(device), seed), torch.device(device))

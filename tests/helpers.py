@@ -98,3 +98,19 @@ def check_routing_fn(B, cfg, ws, inp):
     assert (idx == oidx).all(), "routing indices differ on %d tokens" % (idx != oidx).any(1).sum()
     assert (w.view(np.uint32) == ow.view(np.uint32)).all(), "routing weights differ"
     return L, idx, w, int((gap < NEAR_TIE).sum())
+
+
+def cover_tokens(offs, rows, tile):
+    """Tokens whose rows reach every expert segment and every token tile of
+    the expert GEMMs: for each touched expert its first and last sorted rows,
+    and the last row of each `tile`-row token tile (the ragged tail of every
+    tile the GEMM launches)."""
+    toks = set()
+    for e in range(offs.size - 1):
+        a, b = int(offs[e]), int(offs[e + 1])
+        if b <= a:
+            continue
+        toks.add(int(rows[a]))
+        for t0 in range(a, b, tile):
+            toks.add(int(rows[min(t0 + tile, b) - 1]))
+    return np.array(sorted(toks), dtype=np.int64)

@@ -169,3 +169,29 @@ def test_dsa_calls_reject_bad_arguments_before_launch(B):
     hd = B.DsaConfig(Sq=4, Sk=4, head_dim=64).c()
     st = L.dsa_index_topk(ctypes.byref(hd), 16, 16, None)
     assert st == B.MOE_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments_before_launch(B):
+    """moe_backward validates on the host: fp8 layers, NULL or misaligned
+    buffers and a short workspace are refused before anything is launched."""
+    c = cfg(B)
+    cc = c.c()
+    n = B.backward_workspace_size(c)
+    # the padded row buffers: at least the gathered rows of x and dout, the
+    # gate/up pre-activations and their gradients
+    assert n >= 2 * 64 * 8 * 5120 * 2 + 2 * 64 * 8 * 3072 * 2
+    assert B.backward_workspace_size(cfg(B, T=8192)) > n
+    L = B.lib()
+    p = 1 << 20  # aligned, never dereferenced
+    args = [p] * 17  # x .. dlogits; every call below fails validation, none launches
+    fp8 = cfg(B, dtype=B.MOE_DTYPE_FP8_E4M3_BLOCK128).c()
+    assert L.moe_backward(ctypes.byref(fp8), *args, p, n, None) == B.MOE_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[9] = None  # dout
+    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None) == B.MOE_ERR_INVALID_ARG
+    assert "dout" in B.get_last_error()
+    bad = list(args)
+    bad[10] = p + 2  # dx misaligned
+    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_backward(ctypes.byref(cc), *args, p, n - 256, None) == B.MOE_ERR_WORKSPACE
+    assert L.moe_backward(ctypes.byref(cc), *args, p + 128, n, None) == B.MOE_ERR_INVALID_ARG

@@ -2,8 +2,9 @@
 allocate device memory (a plugin handed only its input and output buffers, a
 runtime whose memory planner owns all of HBM).  Its scratch is a fixed array
 inside the library instead of a caller workspace.  Checked through the C ABI
-against moe_permute (which takes a workspace) on two calls in a row, on the
-single-block and the multi-block paths, and for the size limit.
+against moe_permute (which takes a workspace) and against the oracle's stable
+counting sort, on two calls in a row, on the single-block and the multi-block
+paths, for an empty batch and for the size limit.
 
 Kept in a file of its own that pytest collects last; it also passes alone in
 a fresh process (the first call does the per-device set-up).
@@ -11,6 +12,9 @@ a fresh process (the first call does the per-device set-up).
 import numpy as np
 import pytest
 import torch
+
+from helpers import oracle_cfg
+from oracle import oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +59,19 @@ def test_noalloc_matches_workspace_permute_twice(B, T, E, k):
             assert torch.equal(r, g), "call %d: %s differs" % (call, name)
         offs = got[0].cpu().numpy()
         assert offs[0] == 0 and offs[-1] == T * k and (np.diff(offs) >= 0).all()
+        # the definition: a stable counting sort of the slots by expert
+        for name, o, g in zip(("offsets", "rows", "pos"), O.permute(oracle_cfg(cfg), idx.cpu().numpy()),
+                              got):
+            assert (g.cpu().numpy() == o).all(), "call %d: %s differs from the oracle" % (call, name)
+
+
+def test_noalloc_empty_batch_writes_zero_offsets(B):
+    """T = 0: offsets[0..E] are all zero, as moe_permute writes them."""
+    cfg = B.MoeConfig(T=0, H=512, E=64, k=6, I=128)
+    idx = torch.zeros((1, cfg.k), dtype=torch.int32, device="cuda")
+    ref, got = permute_both(B, cfg, idx)
+    assert torch.equal(ref[0], got[0])
+    assert (got[0] == 0).all()
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(B):
