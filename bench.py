@@ -58,7 +58,11 @@ def parse():
     ap.add_argument("--block", action="store_true",
                     help="time the pre-norm block out = h + MoE(RMSNorm(h)) (moe_forward_block)")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="default decode run: skip the prefill object (T=8192 Zipf) in the line")
+                    help="default decode run: skip the prefill and backward objects (T=8192 "
+                         "Zipf) in the line")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer's backward pass (moe_backward) on the workload instead "
+                         "of the forward")
     return ap.parse_args()
 
 
@@ -795,6 +799,119 @@ def dsa_main(args, world, rank, local):
     dist_teardown(world)
 
 
+# ---------------------------------------------------------------- backward
+
+BWD_METRIC = ("MoE-layer backward tokens/s (gradients of x, router, expert and shared weights) "
+              "and % roofline (bf16 TFLOP/s), 1×B200")
+
+
+def backward_work(wl):
+    """Algorithmic FLOPs of one backward step and of each of its GEMM stages
+    (routed rows T*k; padding rows are overhead, not work)."""
+    T, H, E, k, I, Is = wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is
+    R = T * k
+    st = {"gate_up_recompute": 2 * R * 2 * I * H + 2 * T * 2 * Is * H,
+          "down_backward": 2 * R * H * I + 2 * T * H * Is,
+          "input_grads": 2 * R * 2 * I * H + 2 * T * 2 * Is * H + 2 * T * E * H,
+          "weight_grads": 2 * R * 3 * I * H + 2 * T * 3 * Is * H + 2 * T * E * H}
+    return {"flops": float(sum(st.values())), "stages": st,
+            # weight-gradient outputs (fp32) the step must write
+            "grad_bytes": 4.0 * (E * 3 * H * I + 3 * H * Is + E * H)}
+
+
+def run_backward(args, world, rank, local, inp=None):
+    """Time moe_backward (K steps after W warm-ups, CUDA events on the stream,
+    stage events per launch) on the workload's inputs, routed once by the
+    library's own router outside the timed region."""
+    from sigmoid_top_routing_warp_b200 import binding as B
+    from sigmoid_top_routing_warp_b200 import workloads as W
+    wl = workload_of(args)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    if inp is None:
+        inp = W.make_inputs(wl, device=dev, seed=wl.seed + rank)
+    cfg = cfg_of(B, wl)
+    T, H, E, k, I, Is = wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is
+    stream = torch.cuda.current_stream(dev)
+    ws = B.alloc_workspace(cfg, device=dev)
+    logits = torch.empty((T, E), device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), device=dev)
+    B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], logits, idx, w, ws)
+    dout = W.make_grad_output(wl, device=dev, seed=wl.seed + rank)
+    g = {"dx": torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+         "dwg": torch.empty((E, H), device=dev),
+         "dw13": torch.empty((E, 2 * I, H), device=dev),
+         "dw2": torch.empty((E, H, I), device=dev),
+         "dw13s": torch.empty((2 * Is, H), device=dev) if Is else None,
+         "dw2s": torch.empty((H, Is), device=dev) if Is else None}
+    bws = B.alloc_backward_workspace(cfg, device=dev)
+
+    def step(events=None):
+        B.moe_backward(cfg, inp["x"], inp["w_router"], logits, idx, w, inp["w13"], inp["w2"],
+                       inp["w13s"] if Is else None, inp["w2s"] if Is else None, dout, g["dx"],
+                       g["dwg"], g["dw13"], g["dw2"], g["dw13s"], g["dw2s"], bws,
+                       stream=stream, stage_events=events)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    B.moe_check_device_status(bws)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_NUM_BWD_STAGES + 1)]
+           for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    with ClockSampler(dev.index) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    B.moe_check_device_status(bws)
+    ms = max_over_ranks(world, t0.elapsed_time(t1))
+    stages = np.array([[evs[i][j].elapsed_time(evs[i][j + 1])
+                        for j in range(B.MOE_NUM_BWD_STAGES)] for i in range(K)]).mean(0)
+    touched = int((torch.bincount(idx.flatten().long(), minlength=E) > 0).sum().item())
+    # permute (1 or 3 kernels), plan, gather, 4 GEMMs, router, combine
+    launches = (1 if T * k <= 4096 else 3) + 8
+    return {"wl": wl, "ms": ms, "stage_ms": stages, "clocks": clk.summary(), "touched": touched,
+            "names": B.BWD_STAGE_NAMES, "launches": launches * K}
+
+
+def backward_object(args, rb, peaks, peak_src, world):
+    wl, K = rb["wl"], args.steps
+    work = backward_work(wl)
+    step_ms = rb["ms"] / K
+    stage_ms = {n: float(v) for n, v in zip(rb["names"], rb["stage_ms"])}
+    gemm = {n: stage_ms[n] for n in work["stages"]}
+    dom = max(gemm, key=gemm.get)
+    ach = work["stages"][dom] / (gemm[dom] / 1e3) / 1e12
+    burst = peaks["bf16_tflops"]
+    return {"metric": BWD_METRIC, "value": world * wl.T * K / (rb["ms"] / 1e3), "unit": UNIT,
+            "ms_per_step": step_ms, "tflops": work["flops"] / (step_ms / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s",
+                         "frac": ach / burst, "traffic": None,
+                         "kernel": "bwd_gemm_kernel (%s)" % dom,
+                         "algorithmic_per_launch": work["stages"][dom], "launch_ms": gemm[dom],
+                         "peak_kind": "bf16 burst", "peak_source": peak_src,
+                         "frac_of_sustained_peak":
+                             ach / peaks.get("bf16_tflops_sustained", burst)},
+            "layer_roofline": {"flops": work["flops"],
+                               "t_roof_ms": 1e3 * work["flops"] / (burst * 1e12),
+                               "frac_of_roofline": 1e3 * work["flops"] / (burst * 1e12) / step_ms},
+            "stages_ms": stage_ms, "clocks": rb["clocks"], "gpu_launches": rb["launches"],
+            "experts_touched": rb["touched"], "dtype": "bf16",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+                       "I": wl.I, "n_shared": wl.n_shared, "n_group": wl.n_group,
+                       "topk_group": wl.topk_group, "pass": "backward"}}
+
+
 def routing_check(r):
     """Near-tie count of the timed batch, with the oracle as the checker (part
     of the CPU-baseline leg, outside the timed region): the oracle routes the
@@ -902,6 +1019,18 @@ def main():
         dist_teardown(world)
         return
     peaks, peak_src = load_peaks()
+    if args.backward:
+        rb = run_backward(args, world, rank, local)
+        bo = backward_object(args, rb, peaks, peak_src, world)
+        line = {"metric": bo.pop("metric"), "value": bo.pop("value"), "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": bo.pop("ms_per_step"), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": bo.pop("dtype"),
+                "data": "synthetic", "config": bo.pop("config"), **bo}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        dist_teardown(world)
+        return
     r = run_ours(args, world, rank, local)
     line = layer_line(args, r, peaks, peak_src, world)
     cpu_leg = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -929,6 +1058,12 @@ def main():
             "gpu_launches": pl["gpu_launches"], "routing": pl["routing"]}
         if cpu_leg:
             line["prefill"]["routing"].update(routing_check(rp))
+        # the backward pass of the same prefill batch, on the same inputs
+        inp_p = rp["inp"]
+        del rp
+        torch.cuda.empty_cache()
+        rb = run_backward(pargs, world, rank, local, inp=inp_p)
+        line["backward"] = backward_object(pargs, rb, peaks, peak_src, world)
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist_teardown(world)

@@ -299,6 +299,11 @@ size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
  * the configuration is invalid.                                             */
 size_t moe_backward_workspace_size(const moe_config_t* cfg);
 
+/* Stages of moe_backward: 0 dispatch (permute, padded plan, gather), 1 gate/up
+ * recompute GEMM, 2 down backward GEMM (SwiGLU backward epilogue), 3 router
+ * gradient, 4 input-gradient GEMMs, 5 weight-gradient GEMMs, 6 dx combine. */
+#define MOE_NUM_BWD_STAGES 7
+
 /*   x         bf16 [T, H]        the forward's input
  *   w_router  bf16 [E, H]
  *   logits    fp32 [T, E]        the forward's router logits (moe_route)
@@ -315,6 +320,8 @@ size_t moe_backward_workspace_size(const moe_config_t* cfg);
  *   dlogits   fp32 [T, E]  out   gradient at the router logits, zero off the
  *                                chosen experts; may be NULL
  *   ws        moe_backward_workspace_size bytes
+ *   stage_events  NULL, or MOE_NUM_BWD_STAGES + 1 cudaEvent_t recorded on
+ *             `stream` as the stages start (the last after the last stage)
  * All outputs are overwritten.  Pointers to bf16 data and every output
  * except dlogits must be 16-byte aligned.  fp8 layers return
  * MOE_ERR_UNSUPPORTED.                                                      */
@@ -323,7 +330,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
                           const void* w13, const void* w2, const void* w13s, const void* w2s,
                           const void* dout, void* dx, float* dw_router, float* dw13, float* dw2,
                           float* dw13s, float* dw2s, float* dlogits, void* ws, size_t ws_bytes,
-                          moe_stream_t stream);
+                          void* const* stage_events, moe_stream_t stream);
 
 /* Synchronise `stream`, read the workspace status block of `ws` (the layer's
  * or the DSA indexer's) and clear it.  Returns MOE_OK; MOE_ERR_TIMEOUT if a

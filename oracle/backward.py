@@ -3,7 +3,7 @@ layer: gradients of a loss through the routed SwiGLU experts, the shared
 expert, the renormalised routing weights and the sigmoid router).
 
 TEST INFRASTRUCTURE ONLY, like ``oracle.py``: imported by the test suite,
-never by the product library.  No GPU kernel implements this pass yet.
+never by the product library (whose moe_backward it checks).
 
 What it follows.  The forward pass is the one the pages describe ("Xiaohongshu
 dots3 note Open Source Deep Dive", §3.1 Expert Routing Mechanism: gate ->
@@ -135,3 +135,25 @@ def backward(x, wg, w13, w2, w13s, w2s, idx, dout, norm_topk_prob=True, rsf=1.0)
     dwg = dlogits.T @ x
     return dict(out=out, dx=dx, dwg=dwg, dw13=dw13, dw2=dw2, dw13s=dw13s, dw2s=dw2s, dw=dw,
                 dlogits=dlogits)
+
+
+def expert_grads(x, dout, w, w13, w2):
+    """Weight gradients of ONE SwiGLU expert from the rows that chose it, the
+    chain rule of backward() restricted to that expert (what a full-size check
+    can afford: one expert's weights, not all of them).
+
+    x [n, H] and dout [n, H]: the rows' token inputs and upstream gradients;
+    w [n]: their routing weights (1 for the shared expert, which every token
+    uses); w13 [2I, H] (gate rows, then up rows), w2 [H, I].
+    Returns (dw13 [2I, H], dw2 [H, I])."""
+    I = w13.shape[0] // 2
+    g = x @ w13[:I].T
+    u = x @ w13[I:].T
+    a = _silu(g) * u
+    dy = w[:, None] * dout          # out += w y
+    dw2 = dy.T @ a                  # y = W2 a
+    da = dy @ w2
+    dg = da * u * _dsilu(g)         # a = SiLU(g) u
+    du = da * _silu(g)
+    dw13 = np.concatenate([dg.T @ x, du.T @ x], axis=0)
+    return dw13, dw2

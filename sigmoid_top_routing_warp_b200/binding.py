@@ -24,6 +24,9 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3_BLOCK128 = 1
 MOE_NUM_STAGES = 6
+MOE_NUM_BWD_STAGES = 7
+BWD_STAGE_NAMES = ("dispatch", "gate_up_recompute", "down_backward", "router", "input_grads",
+                   "weight_grads", "combine")
 MOE_FLAG_TEST_STALL = 0x1
 STAGE_NAMES = ("router_gemm", "router_select", "dispatch", "gate_up_swiglu", "down_weighted",
                "combine")
@@ -133,7 +136,7 @@ _lib.moe_quantize_act.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P
 _lib.moe_backward_workspace_size.restype = ctypes.c_size_t
 _lib.moe_backward_workspace_size.argtypes = [_CFG]
 _lib.moe_backward.restype = ctypes.c_int
-_lib.moe_backward.argtypes = [_CFG] + [_P] * 18 + [ctypes.c_size_t, _P]
+_lib.moe_backward.argtypes = [_CFG] + [_P] * 18 + [ctypes.c_size_t, _P, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -289,14 +292,20 @@ def alloc_backward_workspace(cfg: MoeConfig, device="cuda") -> torch.Tensor:
 
 
 def moe_backward(cfg, x, w_router, logits, topk_idx, topk_w, w13, w2, w13s, w2s, dout, dx,
-                 dw_router, dw13, dw2, dw13s, dw2s, ws, dlogits=None, stream=None):
-    """Gradients of sum(out * dout) with the forward's choice held fixed."""
+                 dw_router, dw13, dw2, dw13s, dw2s, ws, dlogits=None, stream=None,
+                 stage_events=None):
+    """Gradients of sum(out * dout) with the forward's choice held fixed.
+    stage_events: None or MOE_NUM_BWD_STAGES + 1 recorded torch.cuda.Event."""
     c = cfg.c()
+    ev = None
+    if stage_events is not None:
+        assert len(stage_events) == MOE_NUM_BWD_STAGES + 1
+        ev = (ctypes.c_void_p * (MOE_NUM_BWD_STAGES + 1))(*[e.cuda_event for e in stage_events])
     _check(_lib.moe_backward(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(logits),
                              _ptr(topk_idx), _ptr(topk_w), _ptr(w13), _ptr(w2), _ptr(w13s),
                              _ptr(w2s), _ptr(dout), _ptr(dx), _ptr(dw_router), _ptr(dw13),
                              _ptr(dw2), _ptr(dw13s), _ptr(dw2s), _ptr(dlogits), _ptr(ws),
-                             ws.numel(), _stream(stream)), "moe_backward")
+                             ws.numel(), ev, _stream(stream)), "moe_backward")
 
 
 def moe_check_device_status(ws, stream=None):

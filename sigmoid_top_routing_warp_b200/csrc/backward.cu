@@ -373,7 +373,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
                           const void* w13, const void* w2, const void* w13s, const void* w2s,
                           const void* dout, void* dx, float* dw_router, float* dw13, float* dw2,
                           float* dw13s, float* dw2s, float* dlogits, void* ws, size_t ws_bytes,
-                          moe_stream_t stream) {
+                          void* const* stage_events, moe_stream_t stream) {
     moe::api_clear_error();
     BW_TRY(moe::api_check_config(cfg));
     if (cfg->dtype != MOE_DTYPE_BF16)
@@ -442,6 +442,14 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
     const int ld_dl = (int)align_up(E, 64);
     int sms = 0;
     BW_TRY(moe::api_sm_count(&sms));
+    cudaEvent_t ev[MOE_NUM_BWD_STAGES + 1] = {};
+    if (stage_events)
+        for (int i = 0; i <= MOE_NUM_BWD_STAGES; ++i) ev[i] = static_cast<cudaEvent_t>(stage_events[i]);
+    auto mark = [&](int i) -> moe_status_t {
+        if (ev[i]) BW_CUDA(cudaEventRecord(ev[i], s), "event record");
+        return MOE_OK;
+    };
+    BW_TRY(mark(0));
 
     // 1. expert segments
     moe::PermuteArgs pa;
@@ -464,6 +472,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
     bwd_gather_kernel<<<(unsigned)((n + E + 7) / 8), 256, 0, s>>>(ga);
     BW_CUDA(cudaGetLastError(), "gather launch");
 
+    BW_TRY(mark(1));
     // 4. G|U = X W13^T (routed, padded rows) and x W13s^T (shared)
     {
         moe::BwdParams P;
@@ -497,6 +506,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         P.status = status;
         BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "gate/up recompute GEMM launch");
     }
+    BW_TRY(mark(2));
     // 5. dA' = dY W2_e with the SwiGLU backward in the epilogue
     {
         moe::BwdParams P;
@@ -543,6 +553,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         P.status = status;
         BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_DSWIGLU, P, sms, s), "down backward GEMM launch");
     }
+    BW_TRY(mark(3));
     // 6. router gradient
     {
         BRouterArgs ra{logits, topk_idx, prow, dwpart, I / 32, dl, ld_dl, dlogits, T, E, k,
@@ -550,6 +561,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         bwd_router_kernel<<<(unsigned)((T + 7) / 8), 256, 0, s>>>(ra);
         BW_CUDA(cudaGetLastError(), "router gradient launch");
     }
+    BW_TRY(mark(4));
     // 7. dX = dG|dU W13_e (routed), dG|dU W13s (shared), dL W_g (router)
     {
         moe::BwdParams P;
@@ -595,6 +607,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         P.status = status;
         BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "input gradient GEMM launch");
     }
+    BW_TRY(mark(5));
     // 8. weight gradients: K = the expert's padded rows (or the T tokens)
     {
         moe::BwdParams P;
@@ -668,6 +681,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         P.status = status;
         BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "weight gradient GEMM launch");
     }
+    BW_TRY(mark(6));
     // 9. dx
     {
         BCombineArgs ca{dxpad, prow, Is > 0 ? dxsh : nullptr, dxr, static_cast<uint16_t*>(dx), T, k, H};
@@ -675,7 +689,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         bwd_combine_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, s>>>(ca);
         BW_CUDA(cudaGetLastError(), "input gradient combine launch");
     }
-    return MOE_OK;
+    return mark(7);
 }
 
 }  // extern "C"

@@ -185,13 +185,13 @@ def test_backward_rejects_bad_arguments_before_launch(B):
     p = 1 << 20  # aligned, never dereferenced
     args = [p] * 17  # x .. dlogits; every call below fails validation, none launches
     fp8 = cfg(B, dtype=B.MOE_DTYPE_FP8_E4M3_BLOCK128).c()
-    assert L.moe_backward(ctypes.byref(fp8), *args, p, n, None) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_backward(ctypes.byref(fp8), *args, p, n, None, None) == B.MOE_ERR_UNSUPPORTED
     bad = list(args)
     bad[9] = None  # dout
-    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None, None) == B.MOE_ERR_INVALID_ARG
     assert "dout" in B.get_last_error()
     bad = list(args)
     bad[10] = p + 2  # dx misaligned
-    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None) == B.MOE_ERR_INVALID_ARG
-    assert L.moe_backward(ctypes.byref(cc), *args, p, n - 256, None) == B.MOE_ERR_WORKSPACE
-    assert L.moe_backward(ctypes.byref(cc), *args, p + 128, n, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_backward(ctypes.byref(cc), *bad, p, n, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_backward(ctypes.byref(cc), *args, p, n - 256, None, None) == B.MOE_ERR_WORKSPACE
+    assert L.moe_backward(ctypes.byref(cc), *args, p + 128, n, None, None) == B.MOE_ERR_INVALID_ARG

@@ -187,3 +187,89 @@ def test_backward_is_deterministic_and_linear(B, W):
     for key, v in z.items():
         if v is not None:
             assert (v == 0).all(), key
+
+
+def test_backward_full_size_prefill(B, W):
+    """The Zipf prefill workload (T = 8192, H = 5120, E = 256, k = 8, I = 1536,
+    one shared expert), sampled where the fp64 oracle can follow it:
+      - dx and dlogits of sampled tokens: the oracle's backward on those
+        tokens with only their experts (a token's dx and dlogits depend on no
+        other token);
+      - dW13_e and dW2_e of the least-loaded, a median and the most-loaded
+        expert (7000+ rows): the oracle's per-expert gradients from the rows
+        that chose the expert, with their routing weights;
+      - dW13s and dW2s over all 8192 tokens (the shared expert, weight 1);
+      - dW_g against dlogits^T x in fp64 from the kernel's own dlogits (a
+        property of that GEMM at full size), within the dot-product error
+        bound of dlogits' bf16 rounding."""
+    wl = W.WORKLOADS["prefill"]
+    inp = W.make_inputs(wl, device="cuda")
+    dout = W.make_grad_output(wl, device="cuda")
+    cfg = mk_cfg(B, wl)
+    T, H, E, k, I, Is = cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.Is
+    dev = "cuda"
+    ws = B.alloc_workspace(cfg)
+    logits = torch.empty((T, E), device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), device=dev)
+    B.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], logits, idx, w, ws)
+    dx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    dwg = torch.empty((E, H), device=dev)
+    dw13 = torch.empty((E, 2 * I, H), device=dev)
+    dw2 = torch.empty((E, H, I), device=dev)
+    dw13s = torch.empty((2 * Is, H), device=dev)
+    dw2s = torch.empty((H, Is), device=dev)
+    dlg = torch.empty((T, E), device=dev)
+    bws = B.alloc_backward_workspace(cfg)
+    B.moe_backward(cfg, inp["x"], inp["w_router"], logits, idx, w, inp["w13"], inp["w2"],
+                   inp["w13s"], inp["w2s"], dout, dx, dwg, dw13, dw2, dw13s, dw2s, bws,
+                   dlogits=dlg)
+    B.moe_check_device_status(bws)
+    idx_h = idx.cpu().numpy().astype(np.int64)
+    w_h = w.cpu().numpy().astype(np.float64)
+
+    # sampled tokens, with only their experts
+    toks = np.array([0, 4321, T - 1])
+    used = np.unique(idx_h[toks])
+    remap = np.full(E, -1, np.int64)
+    remap[used] = np.arange(used.size)
+    sel = torch.as_tensor(used, device=dev)
+    ref = BW.backward(f64(inp["x"][toks]), f64(inp["w_router"][sel]), f64(inp["w13"][sel]),
+                      f64(inp["w2"][sel]), f64(inp["w13s"]), f64(inp["w2s"]),
+                      remap[idx_h[toks]], f64(dout[toks]))
+    assert_close_bf16(f64(dx[toks]), ref["dx"], "prefill dx")
+    assert_close_bf16(f64(dlg[toks][:, sel]), ref["dlogits"], "prefill dlogits")
+    assert (dlg[toks].cpu().numpy()[:, np.setdiff1d(np.arange(E), used)] == 0).all()
+
+    # three experts' weight gradients from the rows that chose them
+    loads = np.bincount(idx_h.ravel(), minlength=E)
+    order = np.argsort(loads, kind="stable")
+    touched = order[loads[order] > 0]
+    for e in (touched[0], touched[touched.size // 2], touched[-1]):
+        t, j = np.nonzero(idx_h == e)
+        ti = torch.as_tensor(t, device=dev)
+        r13, r2 = BW.expert_grads(f64(inp["x"][ti]), f64(dout[ti]), w_h[t, j],
+                                  f64(inp["w13"][int(e)]), f64(inp["w2"][int(e)]))
+        assert_close_grad(f64(dw13[int(e)]), r13, "prefill dw13[%d] (%d rows)" % (e, t.size))
+        assert_close_grad(f64(dw2[int(e)]), r2, "prefill dw2[%d] (%d rows)" % (e, t.size))
+
+    # the shared expert over every token
+    r13s, r2s = BW.expert_grads(f64(inp["x"]), f64(dout), np.ones(T), f64(inp["w13s"]),
+                                f64(inp["w2s"]))
+    assert_close_grad(f64(dw13s), r13s, "prefill dw13s")
+    assert_close_grad(f64(dw2s), r2s, "prefill dw2s")
+
+    # dW_g is dlogits^T x.  Its only rounding is that of dlogits to bf16 (x
+    # is exact, the fp32 accumulation adds ~1e-5 rms), so every element obeys
+    # the dot-product bound |err| <= 2u sum_t |dlogits[t, e] x[t, h]|; an
+    # rms-relative bar does not fit here, where tokens with a small sum of
+    # chosen scores give large terms that cancel
+    x64 = f64(inp["x"])
+    d64 = f64(dlg)
+    ref_g = d64.T @ x64
+    bound = 2 * U_BF16 * (np.abs(d64).T @ np.abs(x64)) + 1e-6 * np.sqrt(np.mean(ref_g ** 2))
+    err = np.abs(f64(dwg) - ref_g)
+    i = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert (err <= bound).all(), "prefill dwg at %s: |err| %.3e > bound %.3e" % (
+        tuple(int(v) for v in i), err[i], bound[i])
+    assert np.linalg.norm(f64(dwg) - ref_g) <= 1e-2 * np.linalg.norm(ref_g)

@@ -135,3 +135,29 @@ def test_backward_is_linear_in_the_upstream_gradient():
     g1, g2, g12 = (BW.backward(*args, d) for d in (d1, d2, d1 + 2.0 * d2))
     for key in ("dx", "dwg", "dw13", "dw2", "dw13s", "dw2s", "dw"):
         assert np.allclose(g12[key], g1[key] + 2.0 * g2[key], rtol=1e-12, atol=1e-12)
+
+
+def test_expert_grads_equal_the_full_backward_per_expert():
+    """expert_grads (one expert's weight gradients from its rows alone) equals
+    backward()'s dw13[e] and dw2[e] for every expert, with the rows' routing
+    weights, and the shared expert's dw13s / dw2s with weight 1 over every
+    token; a dropped routing weight or a swapped gate/up half fails it."""
+    c = small_case(11, T=9, H=16, E=5, k=2, I=6, Is=6)
+    dout = c["rng"].standard_normal((9, 16))
+    ref = BW.backward(c["x"], c["wg"], c["w13"], c["w2"], c["w13s"], c["w2s"], c["idx"], dout)
+    _, cache = BW.forward(c["x"], c["wg"], c["w13"], c["w2"], c["w13s"], c["w2s"], c["idx"])
+    for e in range(5):
+        t, j = np.nonzero(c["idx"] == e)
+        dw13, dw2 = BW.expert_grads(c["x"][t], dout[t], cache["w"][t, j], c["w13"][e], c["w2"][e])
+        assert np.allclose(dw13, ref["dw13"][e], rtol=1e-12, atol=1e-12)
+        assert np.allclose(dw2, ref["dw2"][e], rtol=1e-12, atol=1e-12)
+        if t.size:
+            bad13, bad2 = BW.expert_grads(c["x"][t], dout[t], np.ones(t.size), c["w13"][e],
+                                          c["w2"][e])
+            assert not np.allclose(bad2, ref["dw2"][e])
+            swapped = np.concatenate([c["w13"][e][6:], c["w13"][e][:6]])
+            bad13, _ = BW.expert_grads(c["x"][t], dout[t], cache["w"][t, j], swapped, c["w2"][e])
+            assert not np.allclose(bad13, ref["dw13"][e])
+    dw13s, dw2s = BW.expert_grads(c["x"], dout, np.ones(9), c["w13s"], c["w2s"])
+    assert np.allclose(dw13s, ref["dw13s"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(dw2s, ref["dw2s"], rtol=1e-12, atol=1e-12)
