@@ -285,6 +285,42 @@ moe_status_t moe_forward_block(const moe_config_t* cfg, const void* h, const voi
 size_t moe_workspace_offset(const moe_config_t* cfg, int32_t which);
 
 /* ------------------------------------------------------------------------
+ * Expert parallelism (experts split over ep_size ranks; Deep Dive §8.2
+ * FUSED_MC2 "dispatch -> gmm1 -> swiglu -> gmm2 -> combine" across devices,
+ * §10.2 expert parallelism with an all-to-all backend).  Rank d owns experts
+ * [d E/ep_size, (d+1) E/ep_size).  One rank's step:
+ *   1. moe_route, moe_permute on its own tokens (global expert ids);
+ *   2. moe_ep_pack: its routed rows in expert order, which is destination
+ *      order, with per-destination counts;
+ *   3. all-to-all of counts, then of rows, weights and local expert ids (the
+ *      caller's collective: NCCL over NVLink, or any other);
+ *   4. the received rows are a k = 1 layer over the rank's E/ep_size experts:
+ *      moe_permute, moe_expert_ffn (no shared expert; routed outputs fp32),
+ *      moe_combine back to the receive order;
+ *   5. the reverse all-to-all returns each row to its sender, in its send
+ *      order;
+ *   6. moe_shared_expert and moe_combine on the sender give out.
+ *
+ * moe_ep_pack: for each slot s = t*k + j with sorted row r = pos[s],
+ *   x_send[r] = x[t] (bf16 [T*k, H]), w_send[r] = topk_w[s] (fp32 [T*k]),
+ *   e_send[r] = expert - owner * E/ep_size (int32 [T*k]);
+ *   send_counts[d] = rows for rank d (int32 [ep_size]): the chunk for rank d
+ *   is rows offsets[d E/ep_size] .. offsets[(d+1) E/ep_size] - 1.
+ * ep_size must divide E.  x and x_send 16-byte aligned.                     */
+moe_status_t moe_ep_pack(const moe_config_t* cfg, int32_t ep_size, const void* x,
+                         const int32_t* topk_idx, const float* topk_w, const int32_t* offsets,
+                         const int32_t* pos, void* x_send, float* w_send, int32_t* e_send,
+                         int32_t* send_counts, moe_stream_t stream);
+
+/* The shared expert alone (bf16 layers): y_shared fp32 [T, H] =
+ * SwiGLU_shared(x) with w13s bf16 [2 Is, H], w2s bf16 [H, Is] (Is =
+ * n_shared * I > 0).  ws: moe_workspace_size(cfg) bytes.  Step 6 above; the
+ * pages' "always-on" shared expert (Deep Dive §3.1/§3.3).                    */
+moe_status_t moe_shared_expert(const moe_config_t* cfg, const void* x, const void* w13s,
+                               const void* w2s, float* y_shared, void* ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Backward pass (training side of the layer), bf16 layers.  The pages give
  * the forward pass only (Deep Dive §3.1 gate -> scores -> top-k ->
  * renormalise -> shared + weighted routed sum, §8.2 gmm1 -> swiglu -> gmm2;

@@ -38,7 +38,8 @@ EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", 
             "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
             "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
             "moe_quantize_act", "moe_rmsnorm", "moe_forward_block",
-            "moe_backward_workspace_size", "moe_backward",
+            "moe_backward_workspace_size", "moe_backward", "moe_ep_pack",
+            "moe_shared_expert",
             "dsa_workspace_size", "dsa_workspace_scores_offset", "dsa_index_scores",
             "dsa_index_topk", "dsa_indexer")
 
@@ -137,6 +138,10 @@ _lib.moe_backward_workspace_size.restype = ctypes.c_size_t
 _lib.moe_backward_workspace_size.argtypes = [_CFG]
 _lib.moe_backward.restype = ctypes.c_int
 _lib.moe_backward.argtypes = [_CFG] + [_P] * 18 + [ctypes.c_size_t, _P, _P]
+_lib.moe_ep_pack.restype = ctypes.c_int
+_lib.moe_ep_pack.argtypes = [_CFG, ctypes.c_int32] + [_P] * 10
+_lib.moe_shared_expert.restype = ctypes.c_int
+_lib.moe_shared_expert.argtypes = [_CFG] + [_P] * 5 + [ctypes.c_size_t, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -276,6 +281,23 @@ def moe_quantize_act(x, q, scale, stream=None):
     rows, cols = x.shape
     _check(_lib.moe_quantize_act(_ptr(x), rows, cols, _ptr(q), _ptr(scale), _stream(stream)),
            "moe_quantize_act")
+
+
+def moe_ep_pack(cfg, ep_size, x, topk_idx, topk_w, offsets, pos, x_send, w_send, e_send,
+                send_counts, stream=None):
+    """Expert-parallel send buffer: routed rows in expert (= destination) order."""
+    c = cfg.c()
+    _check(_lib.moe_ep_pack(ctypes.byref(c), int(ep_size), _ptr(x), _ptr(topk_idx),
+                            _ptr(topk_w), _ptr(offsets), _ptr(pos), _ptr(x_send), _ptr(w_send),
+                            _ptr(e_send), _ptr(send_counts), _stream(stream)), "moe_ep_pack")
+
+
+def moe_shared_expert(cfg, x, w13s, w2s, y_shared, ws, stream=None):
+    """The shared expert alone: y_shared (fp32) = SwiGLU_shared(x)."""
+    c = cfg.c()
+    _check(_lib.moe_shared_expert(ctypes.byref(c), _ptr(x), _ptr(w13s), _ptr(w2s),
+                                  _ptr(y_shared), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_shared_expert")
 
 
 def backward_workspace_size(cfg: MoeConfig) -> int:

@@ -699,6 +699,83 @@ moe_status_t run_expert_ffn(const moe_config_t* c, const void* x, const int32_t*
     return MOE_OK;
 }
 
+// The shared expert alone (bf16): y_shared = SwiGLU_shared(x) in fp32, on CTA
+// pairs for prefill-sized batches, single CTAs otherwise.
+moe_status_t run_shared_only(const moe_config_t* c, const void* x, const void* w13s,
+                             const void* w2s, float* y_shared, void* ws, cudaStream_t s) {
+    const Layout L = layout(c);
+    const int Is = c->n_shared * c->I;
+    int sms = 0;
+    MOE_TRY(sm_count(&sms));
+    int* status = at<int>(ws, L.status);
+    void* ash = at<void>(ws, L.ash);
+    if (c->T >= 512) {
+        moe::PairParams P1;
+        memset(&P1, 0, sizeof(P1));
+        moe::PairProblem& q = P1.p[0];
+        MOE_TRY(make_map_gate_up_interleaved(&q.tw, w13s, 1, Is, c->H, "w13s"));
+        MOE_TRY(make_pair_boxes(q.tx, x, c->T, c->H, "x"));
+        q.n_exp = 1;
+        q.n_rows = c->T;
+        q.K = c->H;
+        q.n_feat = Is;
+        q.out = ash;
+        q.ld_out = Is;
+        P1.n_problems = 1;
+        P1.status = status;
+        MOE_CUDA(moe::launch_pair_gemm(moe::EPI_SWIGLU, P1, sms, s), "shared gate/up launch");
+        moe::PairParams P2;
+        memset(&P2, 0, sizeof(P2));
+        moe::PairProblem& r = P2.p[0];
+        MOE_TRY(make_map(&r.tw, w2s, c->H, Is, 128, "w2s"));
+        MOE_TRY(make_pair_boxes(r.tx, ash, c->T, Is, "shared activations"));
+        r.n_exp = 1;
+        r.n_rows = c->T;
+        r.K = Is;
+        r.n_feat = c->H;
+        r.out = y_shared;
+        r.ld_out = c->H;
+        r.out_f32 = 1;
+        P2.n_problems = 1;
+        P2.status = status;
+        MOE_CUDA(moe::launch_pair_gemm(moe::EPI_SCALE, P2, sms, s), "shared down launch");
+        return MOE_OK;
+    }
+    const int bn = c->T <= 16 ? 16 : c->T <= 64 ? 64 : 128;
+    moe::GemmParams P1;
+    memset(&P1, 0, sizeof(P1));
+    moe::GemmProblem& q = P1.p[0];
+    MOE_TRY(make_map(&q.tw, w13s, (size_t)2 * Is, c->H, 128, "w13s"));
+    MOE_TRY(make_map(&q.tx, x, c->T, c->H, bn, "x"));
+    q.n_exp = 1;
+    q.n_rows = c->T;
+    q.K = c->H;
+    q.n_feat = Is;
+    q.w_rows = 2 * Is;
+    q.out = ash;
+    q.ld_out = Is;
+    P1.n_problems = 1;
+    P1.status = status;
+    MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_SWIGLU, bn, P1, sms, s), "shared gate/up launch");
+    moe::GemmParams P2;
+    memset(&P2, 0, sizeof(P2));
+    moe::GemmProblem& r = P2.p[0];
+    MOE_TRY(make_map(&r.tw, w2s, c->H, Is, 128, "w2s"));
+    MOE_TRY(make_map(&r.tx, ash, c->T, Is, bn, "shared activations"));
+    r.n_exp = 1;
+    r.n_rows = c->T;
+    r.K = Is;
+    r.n_feat = c->H;
+    r.w_rows = c->H;
+    r.out = y_shared;
+    r.ld_out = c->H;
+    r.out_f32 = 1;
+    P2.n_problems = 1;
+    P2.status = status;
+    MOE_CUDA(moe::launch_grouped_gemm(moe::EPI_SCALE, bn, P2, sms, s), "shared down launch");
+    return MOE_OK;
+}
+
 moe_status_t check_eps(float eps) {
     if (!(eps >= 0.0f) || !(eps < 1e30f))
         return fail(MOE_ERR_INVALID_ARG, "eps must be finite and >= 0 (got %g)", (double)eps);
@@ -862,6 +939,24 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x, const int32_
     Weights W{w13, w2, w13s, w2s, w13_scale, w2_scale, w13s_scale, w2s_scale};
     return run_expert_ffn(cfg, x, offsets, pos, topk_w, W, y, y_shared, ws,
                           static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+moe_status_t moe_shared_expert(const moe_config_t* cfg, const void* x, const void* w13s,
+                               const void* w2s, float* y_shared, void* ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+    g_err[0] = 0;
+    MOE_TRY(check_config(cfg));
+    if (is_fp8(cfg)) return fail(MOE_ERR_UNSUPPORTED, "moe_shared_expert: bf16 layers only");
+    if (cfg->n_shared < 1) return fail(MOE_ERR_INVALID_ARG, "moe_shared_expert: n_shared is 0");
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    MOE_TRY(need16(x, "x"));
+    MOE_TRY(need16(w13s, "w13s"));
+    MOE_TRY(need16(w2s, "w2s"));
+    MOE_TRY(need16(y_shared, "y_shared"));
+    if (cfg->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    MOE_TRY(reset_claims(ws, s));
+    return run_shared_only(cfg, x, w13s, w2s, y_shared, ws, s);
 }
 
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y, const int32_t* pos,
