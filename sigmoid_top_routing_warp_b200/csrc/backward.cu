@@ -45,6 +45,9 @@ void api_clear_error();
 moe_status_t api_sm_count(int* n);
 moe_status_t api_make_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
                                   uint32_t box_cols, uint32_t box_rows, const char* what);
+moe_status_t api_make_map_3d_bf16(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1,
+                                  uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
+                                  uint32_t b1, uint32_t b2, const char* what);
 }  // namespace moe
 
 namespace {
@@ -354,9 +357,13 @@ using moe::api_make_map_2d_bf16;
 moe_status_t kmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
     return api_make_map_2d_bf16(m, p, rows, cols, 64, 128, what);
 }
-// MN-major operand map: [K rows, MN cols] bf16, box {64, 64}.
+// MN-major operand map of a row-major [K rows, MN cols] bf16 matrix: the 3-D
+// view {64, rows, MN / 64} (strides: a row, 64 elements), box {64, 64, 2}:
+// one copy brings 64 K rows of 128 consecutive MN elements as two 8 KB
+// chunks.  MN is a multiple of 64 for every operand here.
 moe_status_t mnmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
-    return api_make_map_2d_bf16(m, p, rows, cols, 64, 64, what);
+    return moe::api_make_map_3d_bf16(m, p, 64, rows, (cols + 63) / 64, cols * 2, 128, 64, 64, 2,
+                                     what);
 }
 
 }  // namespace

@@ -19,12 +19,18 @@
 // says which), and K may run over an expert's row segment.
 //
 // Tile: 128 x 128 (M = output features in tensor-memory lanes, N = token
-// rows or output columns), K step 64.  Roles (192 threads, one CTA per SM,
+// rows or output columns), K step 64.  Roles (352 threads, one CTA per SM,
 // persistent, static round-robin over the tile list):
-//   warp 0      TMA producer (one 16 KB K-major box, or two 8 KB MN-major
-//               boxes, per operand and stage)
+//   warp 0      TMA producer of the A operand, warp 10 of the B operand: one
+//               16 KB box per operand and stage (a K-major {64, 128} box, or
+//               an MN-major {64, 64, 2} box of a 3-D view that brings both
+//               64-wide chunks); two issuing threads, because one thread's
+//               tensor copies top out well below the SM's L2 bandwidth
 //   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2..5  epilogue (tcgen05.ld 32x32b: lane = feature m)
+//   warps 2..9  epilogue (tcgen05.ld 32x32b: lane = feature m): two warps per
+//               tensor-memory lane quadrant, each taking half of the tile's
+//               columns; stores go through a per-warp shared-memory transpose
+//               so that each thread writes 16 bytes of one output row
 // Two 128-column accumulators let the epilogue of one tile overlap the main
 // loop of the next.  Row segments are padded to 16 rows by the caller, so a
 // segment ends on an MMA boundary: a K step whose 64 rows run past the
@@ -43,7 +49,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kBThreads = 192;
+constexpr int kBEpiWarps = 8;
+constexpr int kBThreads = 32 * (3 + kBEpiWarps);
+constexpr int kBProdB = 2 + kBEpiWarps;           // producer warp of the B operand
 constexpr int kBBK = 64;                          // K per stage
 constexpr int kBT = 128;                          // tile M and N
 constexpr int kBOpBytes = kBT * kBBK * 2;         // 16 KB per operand and stage
@@ -51,7 +59,8 @@ constexpr int kBStage = 2 * kBOpBytes;
 constexpr int kBStages = 6;
 constexpr uint32_t kBChunk = kBBK * 128;          // one 64-wide MN chunk: 64 K rows x 128 B
 constexpr int kBBarBytes = 256;
-constexpr int kBSmem = 1024 + kBStages * kBStage + kBBarBytes;
+constexpr int kBEpiBytes = kBEpiWarps * 32 * 32 * 4;  // per-warp [32 columns][32 features] fp32
+constexpr int kBSmem = 1024 + kBStages * kBStage + kBEpiBytes + kBBarBytes;
 constexpr int kBTmemCols = 2 * kBT;
 static_assert(kBSmem <= 232448, "shared memory budget");
 
@@ -128,16 +137,16 @@ __device__ __forceinline__ int bk_blocks(const BTile& t) {
     return t.k1 > t.k0 ? (t.k1 - t.k0 + kBBK - 1) / kBBK : 0;
 }
 
-// One operand of one stage: a K-major box {64 K, 128 rows} at (k, row0 + mn0),
-// or two MN-major boxes {64 MN, 64 K} at (mn0 (+64), row0 + k).
+// One operand of one stage: a K-major box {64 K, 128 rows} at (k, row0 + mn0)
+// of a 2-D map, or an MN-major box {64, 64 K, 2 chunks} at (0, row0 + k,
+// mn0 / 64) of the 3-D view {64, rows, MN / 64} (chunk c lands kBChunk bytes
+// after chunk c - 1).
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* m, int mn_major,
                                              int mn0, int k, int row0, uint64_t* bar) {
-    if (!mn_major) {
+    if (!mn_major)
         tma_load_2d(dst, m, bar, k, row0 + mn0);
-    } else {
-        tma_load_2d(dst, m, bar, mn0, row0 + k);
-        tma_load_2d(dst + kBChunk, m, bar, mn0 + 64, row0 + k);
-    }
+    else
+        tma_load_3d(dst, m, bar, 0, row0 + k, mn0 >> 6);
 }
 
 // Descriptor of the 16-deep K slice kk of an operand stage.
@@ -157,7 +166,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBStages * kBStage);
+    float* epi_smem = reinterpret_cast<float*>(smem + kBStages * kBStage);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBStages * kBStage + kBEpiBytes);
     uint64_t* empty = full + kBStages;
     uint64_t* tfull = empty + kBStages;
     uint64_t* tempty = tfull + 2;
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], kBEpiWarps);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -195,9 +205,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = btotal(P);
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    if (warp == 0 || warp == kBProdB) {
+        // ------------------------------------------------ TMA producers
+        // Warp 0 loads A and sets the stage's expected bytes (both operands);
+        // warp kBProdB loads B.  A copy that lands before the expectation is
+        // set leaves the barrier's phase open: warp 0's arrival is pending.
         if (lane == 0) {
+            const bool pa = warp == 0;
             int s = 0;
             uint32_t ph = 0, issued = 0, last_ph = 0;
             bool ok = true;
@@ -211,17 +225,22 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                     if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
                     uint8_t* st = smem + s * kBStage;
                     const int k = tl.k0 + kb * kBBK;
-                    mbar_arrive_expect_tx(&full[s], kBStage);
-                    load_operand(st, &p.ta, p.a_mn, tl.m0, k, arow, &full[s]);
-                    load_operand(st + kBOpBytes, &p.tb, p.b_mn, tl.n0, k, 0, &full[s]);
+                    if (pa) {
+                        mbar_arrive_expect_tx(&full[s], kBStage);
+                        load_operand(st, &p.ta, p.a_mn, tl.m0, k, arow, &full[s]);
+                    } else {
+                        load_operand(st + kBOpBytes, &p.tb, p.b_mn, tl.n0, k, 0, &full[s]);
+                    }
                     issued |= 1u << s;
                     last_ph = (last_ph & ~(1u << s)) | (ph << s);
                     if (++s == kBStages) { s = 0; ph ^= 1; }
                 }
             }
-            // leave no copy in flight
-            for (int i = 0; i < kBStages; ++i)
-                if (issued >> i & 1u) wait_bar(&full[i], last_ph >> i & 1u, abort_flag, P.status, true);
+            // leave no copy in flight: warp 0 waits for the last fill of every
+            // stage, which counts both producers' copies
+            if (pa)
+                for (int i = 0; i < kBStages; ++i)
+                    if (issued >> i & 1u) wait_bar(&full[i], last_ph >> i & 1u, abort_flag, P.status, true);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -273,7 +292,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // tensor-memory lane quadrant of this warp
+        const int q = warp & 3;           // tensor-memory lane quadrant of this warp
+        const int half = (warp - 2) >> 2;  // columns [64 half, 64 half + 64) of a tile
+        float* stg = epi_smem + (warp - 2) * 32 * 32;
         int buf = 0;
         uint32_t aph = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -286,9 +307,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
             const int m = tl.m0 + q * 32 + lane;
             const bool mok = m < p.M;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kBT;
+            const int cend = min(tl.nvalid, 64 * half + 64);
             if (EPI == BEPI_STORE) {
                 const size_t obase = (size_t)tl.grp * (size_t)p.out_grp;
-                for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
+                const int mq = tl.m0 + q * 32;  // first feature of this warp's 32
+                for (int c0 = 64 * half; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);
@@ -297,19 +320,39 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
 #pragma unroll
                         for (int j = 0; j < 32; ++j) r[j] = 0u;
                     }
+                    // transpose: stg[column j][feature lane]
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __uint_as_float(r[j]);
+                    __syncwarp();
                     if (p.out_f32) {
+                        // 8 lanes write one column's 32 features (128 B) as 16-byte chunks
                         float* out = reinterpret_cast<float*>(p.out) + obase;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (c0 + j < tl.nvalid && mok)
-                                out[(size_t)(tl.n0 + c0 + j) * p.ld_out + m] = __uint_as_float(r[j]);
+                        for (int it = 0; it < 8; ++it) {
+                            const int row = 4 * it + (lane >> 3), ch = lane & 7;
+                            if (c0 + row < tl.nvalid && mq + 4 * ch < p.M)
+                                *reinterpret_cast<float4*>(out + (size_t)(tl.n0 + c0 + row) * p.ld_out +
+                                                           mq + 4 * ch) =
+                                    *reinterpret_cast<const float4*>(stg + row * 32 + 4 * ch);
+                        }
                     } else {
+                        // 4 lanes write one column's 32 features (64 B) as 8 bf16 each
                         uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + obase;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (c0 + j < tl.nvalid && mok)
-                                out[(size_t)(tl.n0 + c0 + j) * p.ld_out + m] = f2bf(__uint_as_float(r[j]));
+                        for (int it = 0; it < 4; ++it) {
+                            const int row = 8 * it + (lane >> 2), ch = lane & 3;
+                            if (c0 + row < tl.nvalid && mq + 8 * ch < p.M) {
+                                const float* v = stg + row * 32 + 8 * ch;
+                                uint32_t w4[4];
+#pragma unroll
+                                for (int h = 0; h < 4; ++h)
+                                    w4[h] = (uint32_t)f2bf(v[2 * h]) | ((uint32_t)f2bf(v[2 * h + 1]) << 16);
+                                *reinterpret_cast<uint4*>(out + (size_t)(tl.n0 + c0 + row) * p.ld_out +
+                                                          mq + 8 * ch) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            }
+                        }
                     }
+                    __syncwarp();
                 }
             } else {
                 // SwiGLU backward for 128 features i (lanes) of 32 rows at a
@@ -318,7 +361,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                 //   dg = da u sigma(g) (1 + g (1 - sigma(g))),  du = da SiLU(g),
                 // and the routing-weight gradient's partial sum over this
                 // warp's 32 features, sum_i a_i da'_i.
-                for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
+                for (int c0 = 64 * half; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);

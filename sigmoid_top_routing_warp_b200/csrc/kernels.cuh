@@ -202,8 +202,8 @@ cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cuda
 // One problem of a backward grouped GEMM launch (gemm_bwd.cu).  The tensor-
 // memory accumulator of a tile is D[m, n] = sum_k A(m, k) B(n, k) over a
 // 128 x 128 tile, lane = m, column = n; each operand is K-major (a 2-D map
-// [rows, K], box {64, 128}) or MN-major (a 2-D map [K, MN], box {64, 64},
-// two boxes per stage).
+// [rows, K], box {64, 128}) or MN-major (a 3-D view {64, K rows, MN / 64} of
+// the row-major [K, MN] matrix, strides {MN * 2, 128} bytes, box {64, 64, 2}).
 //   rows_as_k = 0: the N dimension runs over token rows, grouped by `seg`
 //     (per group: tiles of 128 rows, prefix `tstart`), K = [0, K); A's row
 //     coordinate is offset by group * a_grp_rows (the group's weights).
