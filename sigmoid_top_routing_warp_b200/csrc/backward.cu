@@ -16,7 +16,7 @@
 //
 // Sequence on one stream:
 //   1. permute (as the forward) -> expert segments
-//   2. plan: segments padded to 16 rows (pstart) and their 128-row tile
+//   2. plan: segments padded to 16 rows (pstart) and their 256-row tile
 //      prefix (tstart); a weight-gradient GEMM contracts over a padded
 //      segment, and 16 rows is one MMA's K
 //   3. gather: X and dout rows into the padded order, routing weight per
@@ -53,7 +53,7 @@ moe_status_t api_make_map_3d_bf16(CUtensorMap* m, const void* ptr, uint64_t d0, 
 namespace {
 
 constexpr int kPadRows = 16;   // segment padding: one MMA's K
-constexpr int kRowTile = 128;  // token rows per tile of the rows-as-N GEMMs
+constexpr int kRowTile = 256;  // token rows per tile of the rows-as-N GEMMs
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -136,7 +136,7 @@ moe_status_t bcuda(cudaError_t e, const char* what) {
 struct PlanArgs {
     const int32_t* offsets;
     int32_t* pstart;  // [E + 1] padded segment starts
-    int32_t* tstart;  // [E + 1] prefix of 128-row tiles over the padded segments
+    int32_t* tstart;  // [E + 1] prefix of 256-row tiles over the padded segments
     int E;
 };
 
@@ -353,9 +353,12 @@ moe_status_t need16(const void* p, const char* name) {
 
 using moe::api_make_map_2d_bf16;
 
-// K-major operand map: [rows, cols] bf16, box {64, 128}.
+// K-major operand maps: [rows, cols] bf16, box {64, 128} (A) or {64, 256} (B).
 moe_status_t kmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
     return api_make_map_2d_bf16(m, p, rows, cols, 64, 128, what);
+}
+moe_status_t kmapB(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
+    return api_make_map_2d_bf16(m, p, rows, cols, 64, 256, what);
 }
 // MN-major operand map of a row-major [K rows, MN cols] bf16 matrix: the 3-D
 // view {64, rows, MN / 64} (strides: a row, 64 elements), box {64, 64, 2}:
@@ -363,6 +366,11 @@ moe_status_t kmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const
 // chunks.  MN is a multiple of 64 for every operand here.
 moe_status_t mnmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
     return moe::api_make_map_3d_bf16(m, p, 64, rows, (cols + 63) / 64, cols * 2, 128, 64, 64, 2,
+                                     what);
+}
+// The same for a B operand: box {64, 64, 4}, 256 consecutive MN elements.
+moe_status_t mnmapB(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
+    return moe::api_make_map_3d_bf16(m, p, 64, rows, (cols + 63) / 64, cols * 2, 128, 64, 64, 4,
                                      what);
 }
 
@@ -486,7 +494,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         memset(&P, 0, sizeof(P));
         moe::BwdProblem& p = P.p[0];
         BW_TRY(kmap(&p.ta, w13, (size_t)E * 2 * I, H, "w13"));
-        BW_TRY(kmap(&p.tb, xpad, R, H, "padded x"));
+        BW_TRY(kmapB(&p.tb, xpad, R, H, "padded x"));
+        BW_TRY(kmap(&p.tb_half, xpad, R, H, "padded x"));
         p.seg = pstart;
         p.tstart = tstart;
         p.n_grp = E;
@@ -500,7 +509,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[1];
             BW_TRY(kmap(&q.ta, w13s, (size_t)2 * Is, H, "w13s"));
-            BW_TRY(kmap(&q.tb, x, T, H, "x"));
+            BW_TRY(kmapB(&q.tb, x, T, H, "x"));
+            BW_TRY(kmap(&q.tb_half, x, T, H, "x"));
             q.n_grp = 1;
             q.n_rows = T;
             q.M = 2 * Is;
@@ -520,7 +530,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         memset(&P, 0, sizeof(P));
         moe::BwdProblem& p = P.p[0];
         BW_TRY(mnmap(&p.ta, w2, (size_t)E * H, I, "w2"));
-        BW_TRY(kmap(&p.tb, dypad, R, H, "padded dout"));
+        BW_TRY(kmapB(&p.tb, dypad, R, H, "padded dout"));
+        BW_TRY(kmap(&p.tb_half, dypad, R, H, "padded dout"));
         p.a_mn = 1;
         p.seg = pstart;
         p.tstart = tstart;
@@ -542,7 +553,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[1];
             BW_TRY(mnmap(&q.ta, w2s, H, Is, "w2s"));
-            BW_TRY(kmap(&q.tb, dout, T, H, "dout"));
+            BW_TRY(kmapB(&q.tb, dout, T, H, "dout"));
+            BW_TRY(kmap(&q.tb_half, dout, T, H, "dout"));
             q.a_mn = 1;
             q.n_grp = 1;
             q.n_rows = T;
@@ -576,7 +588,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         int np = 0;
         moe::BwdProblem& p = P.p[np++];
         BW_TRY(mnmap(&p.ta, w13, (size_t)E * 2 * I, H, "w13"));
-        BW_TRY(kmap(&p.tb, dgu, R, 2 * I, "padded dgate/dup"));
+        BW_TRY(kmapB(&p.tb, dgu, R, 2 * I, "padded dgate/dup"));
+        BW_TRY(kmap(&p.tb_half, dgu, R, 2 * I, "padded dgate/dup"));
         p.a_mn = 1;
         p.seg = pstart;
         p.tstart = tstart;
@@ -589,7 +602,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[np++];
             BW_TRY(mnmap(&q.ta, w13s, (size_t)2 * Is, H, "w13s"));
-            BW_TRY(kmap(&q.tb, dgus, T, 2 * Is, "shared dgate/dup"));
+            BW_TRY(kmapB(&q.tb, dgus, T, 2 * Is, "shared dgate/dup"));
+            BW_TRY(kmap(&q.tb_half, dgus, T, 2 * Is, "shared dgate/dup"));
             q.a_mn = 1;
             q.n_grp = 1;
             q.n_rows = T;
@@ -601,7 +615,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         }
         moe::BwdProblem& r = P.p[np++];
         BW_TRY(mnmap(&r.ta, w_router, E, H, "w_router"));
-        BW_TRY(kmap(&r.tb, dl, T, ld_dl, "router dlogits"));
+        BW_TRY(kmapB(&r.tb, dl, T, ld_dl, "router dlogits"));
+        BW_TRY(kmap(&r.tb_half, dl, T, ld_dl, "router dlogits"));
         r.a_mn = 1;
         r.n_grp = 1;
         r.n_rows = T;
@@ -622,7 +637,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         int np = 0;
         moe::BwdProblem& p = P.p[np++];  // dW2_e[h][i] = sum_r dY[r][h] (w a)[r][i]
         BW_TRY(mnmap(&p.ta, aw, R, I, "padded w*a"));
-        BW_TRY(mnmap(&p.tb, dypad, R, H, "padded dout"));
+        BW_TRY(mnmapB(&p.tb, dypad, R, H, "padded dout"));
         p.a_mn = p.b_mn = 1;
         p.rows_as_k = 1;
         p.seg = pstart;
@@ -635,7 +650,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         p.out_f32 = 1;
         moe::BwdProblem& q = P.p[np++];  // dW13_e[j][h] = sum_r dGU[r][j] X[r][h]
         BW_TRY(mnmap(&q.ta, xpad, R, H, "padded x"));
-        BW_TRY(mnmap(&q.tb, dgu, R, 2 * I, "padded dgate/dup"));
+        BW_TRY(mnmapB(&q.tb, dgu, R, 2 * I, "padded dgate/dup"));
         q.a_mn = q.b_mn = 1;
         q.rows_as_k = 1;
         q.seg = pstart;
@@ -649,7 +664,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& a2 = P.p[np++];  // dW2s[h][i]
             BW_TRY(mnmap(&a2.ta, as, T, Is, "shared a"));
-            BW_TRY(mnmap(&a2.tb, dout, T, H, "dout"));
+            BW_TRY(mnmapB(&a2.tb, dout, T, H, "dout"));
             a2.a_mn = a2.b_mn = 1;
             a2.rows_as_k = 1;
             a2.n_grp = 1;
@@ -661,7 +676,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
             a2.out_f32 = 1;
             moe::BwdProblem& a3 = P.p[np++];  // dW13s[j][h]
             BW_TRY(mnmap(&a3.ta, x, T, H, "x"));
-            BW_TRY(mnmap(&a3.tb, dgus, T, 2 * Is, "shared dgate/dup"));
+            BW_TRY(mnmapB(&a3.tb, dgus, T, 2 * Is, "shared dgate/dup"));
             a3.a_mn = a3.b_mn = 1;
             a3.rows_as_k = 1;
             a3.n_grp = 1;
@@ -674,7 +689,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         }
         moe::BwdProblem& g = P.p[np++];  // dW_g[e][h] = sum_t dL[t][e] x[t][h]
         BW_TRY(mnmap(&g.ta, x, T, H, "x"));
-        BW_TRY(mnmap(&g.tb, dl, T, ld_dl, "router dlogits"));
+        BW_TRY(mnmapB(&g.tb, dl, T, ld_dl, "router dlogits"));
         g.a_mn = g.b_mn = 1;
         g.rows_as_k = 1;
         g.n_grp = 1;

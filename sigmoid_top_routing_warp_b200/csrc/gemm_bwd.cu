@@ -18,21 +18,22 @@
 // tensor core reads either from shared memory; the instruction descriptor
 // says which), and K may run over an expert's row segment.
 //
-// Tile: 128 x 128 (M = output features in tensor-memory lanes, N = token
-// rows or output columns), K step 64.  Roles (352 threads, one CTA per SM,
+// Tile: 128 x 256 (M = output features in tensor-memory lanes, N = token
+// rows or output columns), K step 64; the MMA's N is the tile's valid
+// columns rounded up to 16.  Roles (352 threads, one CTA per SM,
 // persistent, static round-robin over the tile list):
-//   warp 0      TMA producer of the A operand, warp 10 of the B operand: one
-//               16 KB box per operand and stage (a K-major {64, 128} box, or
-//               an MN-major {64, 64, 2} box of a 3-D view that brings both
-//               64-wide chunks); two issuing threads, because one thread's
+//   warp 0      TMA producer of the A operand (one 16 KB box per stage: K-major
+//               {64, 128}, or MN-major {64, 64, 2} of a 3-D view that brings
+//               two 64-wide chunks), warp 10 of the B operand (32 KB: {64, 256}
+//               or {64, 64, 4}); two issuing threads, because one thread's
 //               tensor copies top out well below the SM's L2 bandwidth
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //   warps 2..9  epilogue (tcgen05.ld 32x32b: lane = feature m): two warps per
 //               tensor-memory lane quadrant, each taking half of the tile's
 //               columns; stores go through a per-warp shared-memory transpose
 //               so that each thread writes 16 bytes of one output row
-// Two 128-column accumulators let the epilogue of one tile overlap the main
-// loop of the next.  Row segments are padded to 16 rows by the caller, so a
+// Two 256-column accumulators (all of tensor memory) let the epilogue of one
+// tile overlap the main loop of the next.  Row segments are padded to 16 rows by the caller, so a
 // segment ends on an MMA boundary: a K step whose 64 rows run past the
 // segment issues only the MMAs inside it.
 //
@@ -53,15 +54,17 @@ constexpr int kBEpiWarps = 8;
 constexpr int kBThreads = 32 * (3 + kBEpiWarps);
 constexpr int kBProdB = 2 + kBEpiWarps;           // producer warp of the B operand
 constexpr int kBBK = 64;                          // K per stage
-constexpr int kBT = 128;                          // tile M and N
-constexpr int kBOpBytes = kBT * kBBK * 2;         // 16 KB per operand and stage
-constexpr int kBStage = 2 * kBOpBytes;
-constexpr int kBStages = 6;
+constexpr int kBT = 128;                          // tile M (tensor-memory lanes)
+constexpr int kBN = 256;                          // tile N (columns)
+constexpr int kBABytes = kBT * kBBK * 2;          // 16 KB of A per stage
+constexpr int kBBBytes = kBN * kBBK * 2;          // 32 KB of B per stage
+constexpr int kBStage = kBABytes + kBBBytes;
+constexpr int kBStages = 4;
 constexpr uint32_t kBChunk = kBBK * 128;          // one 64-wide MN chunk: 64 K rows x 128 B
 constexpr int kBBarBytes = 256;
 constexpr int kBEpiBytes = kBEpiWarps * 32 * 32 * 4;  // per-warp [32 columns][32 features] fp32
 constexpr int kBSmem = 1024 + kBStages * kBStage + kBEpiBytes + kBBarBytes;
-constexpr int kBTmemCols = 2 * kBT;
+constexpr int kBTmemCols = 2 * kBN;
 static_assert(kBSmem <= 232448, "shared memory budget");
 
 struct BTile {
@@ -70,8 +73,8 @@ struct BTile {
 
 __device__ __forceinline__ int bprob_tiles(const BwdProblem& p) {
     const int mt = (p.M + kBT - 1) / kBT;
-    if (p.rows_as_k) return p.n_grp * mt * ((p.N + kBT - 1) / kBT);
-    if (p.seg == nullptr) return mt * ((p.n_rows + kBT - 1) / kBT);
+    if (p.rows_as_k) return p.n_grp * mt * ((p.N + kBN - 1) / kBN);
+    if (p.seg == nullptr) return mt * ((p.n_rows + kBN - 1) / kBN);
     return mt * __ldg(p.tstart + p.n_grp);
 }
 
@@ -94,21 +97,21 @@ __device__ __forceinline__ bool btile_at(const BwdParams& P, int t, BTile& o) {
         const int mt = (p.M + kBT - 1) / kBT;
         o.prob = pi;
         if (p.rows_as_k) {
-            const int nt = (p.N + kBT - 1) / kBT;
+            const int nt = (p.N + kBN - 1) / kBN;
             const int g = t / (mt * nt);
             const int l = t - g * mt * nt;
             o.grp = g;
             o.m0 = (l / nt) * kBT;
-            o.n0 = (l % nt) * kBT;
-            o.nvalid = min(kBT, p.N - o.n0);
+            o.n0 = (l % nt) * kBN;
+            o.nvalid = min(kBN, p.N - o.n0);
             o.k0 = p.seg ? __ldg(p.seg + g) : 0;
             o.k1 = p.seg ? __ldg(p.seg + g + 1) : p.n_rows;
         } else if (p.seg == nullptr) {
-            const int nt = (p.n_rows + kBT - 1) / kBT;
+            const int nt = (p.n_rows + kBN - 1) / kBN;
             o.grp = 0;
             o.m0 = (t / nt) * kBT;
-            o.n0 = (t % nt) * kBT;
-            o.nvalid = min(kBT, p.n_rows - o.n0);
+            o.n0 = (t % nt) * kBN;
+            o.nvalid = min(kBN, p.n_rows - o.n0);
             o.k0 = 0;
             o.k1 = p.K;
         } else {
@@ -123,8 +126,8 @@ __device__ __forceinline__ bool btile_at(const BwdParams& P, int t, BTile& o) {
             const int ntg = __ldg(p.tstart + g + 1) - __ldg(p.tstart + g);
             o.grp = g;
             o.m0 = (l / ntg) * kBT;
-            o.n0 = __ldg(p.seg + g) + (l % ntg) * kBT;
-            o.nvalid = min(kBT, __ldg(p.seg + g + 1) - o.n0);
+            o.n0 = __ldg(p.seg + g) + (l % ntg) * kBN;
+            o.nvalid = min(kBN, __ldg(p.seg + g + 1) - o.n0);
             o.k0 = 0;
             o.k1 = p.K;
         }
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
         for (int pi = 0; pi < P.n_problems; ++pi) {
             tma_prefetch_desc(&P.p[pi].ta);
             tma_prefetch_desc(&P.p[pi].tb);
+            if (!P.p[pi].rows_as_k && !P.p[pi].b_mn) tma_prefetch_desc(&P.p[pi].tb_half);
         }
     }
     if (warp == 1) {
@@ -221,15 +225,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                 const BwdProblem& p = P.p[tl.prob];
                 const int nkb = bk_blocks(tl);
                 const int arow = p.rows_as_k ? 0 : tl.grp * p.a_grp_rows;
+                // a row tile with at most 128 valid rows loads a 128-row B box
+                const bool bhalf = !p.rows_as_k && !p.b_mn && tl.nvalid <= kBN / 2;
+                const uint32_t stage_bytes = kBABytes + (bhalf ? kBBBytes / 2 : kBBBytes);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
                     uint8_t* st = smem + s * kBStage;
                     const int k = tl.k0 + kb * kBBK;
                     if (pa) {
-                        mbar_arrive_expect_tx(&full[s], kBStage);
+                        mbar_arrive_expect_tx(&full[s], stage_bytes);
                         load_operand(st, &p.ta, p.a_mn, tl.m0, k, arow, &full[s]);
                     } else {
-                        load_operand(st + kBOpBytes, &p.tb, p.b_mn, tl.n0, k, 0, &full[s]);
+                        load_operand(st + kBABytes, bhalf ? &p.tb_half : &p.tb, p.b_mn, tl.n0, k, 0,
+                                     &full[s]);
                     }
                     issued |= 1u << s;
                     last_ph = (last_ph & ~(1u << s)) | (ph << s);
@@ -254,10 +262,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                 btile_at(P, t, tl);
                 const BwdProblem& p = P.p[tl.prob];
                 const int nkb = bk_blocks(tl);
-                const uint32_t idesc = idesc_bf16_f32_major(kBT, kBT, p.a_mn, p.b_mn);
+                // N: the tile's valid columns rounded up to 16 (an M = 128 MMA
+                // takes N in steps of 16), so a ragged row tile pays only for its rows
+                const uint32_t idesc = idesc_bf16_f32_major(kBT, min(kBN, (tl.nvalid + 15) & ~15),
+                                                            p.a_mn, p.b_mn);
                 if (!wait_bar(&tempty[buf], aph ^ 1, abort_flag, P.status)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + buf * kBT;
+                const uint32_t d = tmem_base + buf * kBN;
                 bool first = true;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!wait_bar(&full[s], ph, abort_flag, P.status)) { ok = false; break; }
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
 #pragma unroll
                     for (int kk = 0; kk < kBBK / 16; ++kk) {
                         if (16 * kk < krem) {
-                            tc_mma_f16(d, op_desc(st, p.a_mn, kk), op_desc(st + kBOpBytes, p.b_mn, kk),
+                            tc_mma_f16(d, op_desc(st, p.a_mn, kk), op_desc(st + kBABytes, p.b_mn, kk),
                                        idesc, first ? 0u : 1u);
                             first = false;
                         }
@@ -306,12 +317,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
             const bool has_k = bk_blocks(tl) > 0;
             const int m = tl.m0 + q * 32 + lane;
             const bool mok = m < p.M;
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kBT;
-            const int cend = min(tl.nvalid, 64 * half + 64);
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kBN;
+            const int cend = min(tl.nvalid, (kBN / 2) * half + kBN / 2);
             if (EPI == BEPI_STORE) {
                 const size_t obase = (size_t)tl.grp * (size_t)p.out_grp;
                 const int mq = tl.m0 + q * 32;  // first feature of this warp's 32
-                for (int c0 = 64 * half; c0 < cend; c0 += 32) {
+                for (int c0 = (kBN / 2) * half; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);
@@ -361,7 +372,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                 //   dg = da u sigma(g) (1 + g (1 - sigma(g))),  du = da SiLU(g),
                 // and the routing-weight gradient's partial sum over this
                 // warp's 32 features, sum_i a_i da'_i.
-                for (int c0 = 64 * half; c0 < cend; c0 += 32) {
+                for (int c0 = (kBN / 2) * half; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);
@@ -380,7 +391,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                             const float g = p.gu[(size_t)row * p.ld_gu + m];
                             const float u = p.gu[(size_t)row * p.ld_gu + p.half + m];
                             const float w = p.row_w ? __ldg(p.row_w + row) : 1.0f;
-                            const float sg = 1.0f / (1.0f + __expf(-g));
+                            const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
                             const float sl = g * sg;
                             const float a = sl * u;
                             const float da = w * da1;
