@@ -382,25 +382,37 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                         for (int j = 0; j < 32; ++j) r[j] = 0u;
                     }
                     float part[32];
+                    // eight rows at a time: their pre-activations and weights are
+                    // loaded (read-only path) before any of the eight rows' stores
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        part[j] = 0.0f;
-                        const int row = tl.n0 + c0 + j;
-                        if (c0 + j < tl.nvalid && mok) {
-                            const float da1 = __uint_as_float(r[j]);
-                            const float g = p.gu[(size_t)row * p.ld_gu + m];
-                            const float u = p.gu[(size_t)row * p.ld_gu + p.half + m];
-                            const float w = p.row_w ? __ldg(p.row_w + row) : 1.0f;
-                            const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
-                            const float sl = g * sg;
-                            const float a = sl * u;
-                            const float da = w * da1;
-                            const float dg = da * u * sg * (1.0f + g * (1.0f - sg));
-                            const float du = da * sl;
-                            p.dgu[(size_t)row * p.ld_dgu + m] = f2bf(dg);
-                            p.dgu[(size_t)row * p.ld_dgu + p.half + m] = f2bf(du);
-                            p.aw[(size_t)row * p.ld_aw + m] = f2bf(w * a);
-                            part[j] = a * da1;
+                    for (int j0 = 0; j0 < 32; j0 += 8) {
+                        float gv[8], uv[8], wv[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int row = tl.n0 + c0 + j0 + j;
+                            const bool ok_rc = c0 + j0 + j < tl.nvalid && mok;
+                            gv[j] = ok_rc ? __ldg(p.gu + (size_t)row * p.ld_gu + m) : 0.0f;
+                            uv[j] = ok_rc ? __ldg(p.gu + (size_t)row * p.ld_gu + p.half + m) : 0.0f;
+                            wv[j] = (ok_rc && p.row_w) ? __ldg(p.row_w + row) : 1.0f;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int row = tl.n0 + c0 + j0 + j;
+                            part[j0 + j] = 0.0f;
+                            if (c0 + j0 + j < tl.nvalid && mok) {
+                                const float da1 = __uint_as_float(r[j0 + j]);
+                                const float g = gv[j], u = uv[j], w = wv[j];
+                                const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+                                const float sl = g * sg;
+                                const float a = sl * u;
+                                const float da = w * da1;
+                                const float dg = da * u * sg * (1.0f + g * (1.0f - sg));
+                                const float du = da * sl;
+                                p.dgu[(size_t)row * p.ld_dgu + m] = f2bf(dg);
+                                p.dgu[(size_t)row * p.ld_dgu + p.half + m] = f2bf(du);
+                                p.aw[(size_t)row * p.ld_aw + m] = f2bf(w * a);
+                                part[j0 + j] = a * da1;
+                            }
                         }
                     }
                     if (p.dw_part) {
