@@ -249,14 +249,20 @@ def profile_traffic(kind, algorithmic, workload):
                         records.append({})
                     if records:
                         records[-1][k] = v.strip()
+    generic = None
     for fields in records:
         if fields.get("kernel") != kind or fields.get("source_hash") != source_hash(kind):
             continue
         # a capture of this exact workload wins over a ratio scaled from a smaller case
         if "traffic_bytes_per_launch" in fields and fields.get("workload") == workload:
             return float(fields["traffic_bytes_per_launch"])
-        if "traffic_over_algorithmic" in fields and ratio is None:
-            ratio = float(fields["traffic_over_algorithmic"])
+        if "traffic_over_algorithmic" in fields:
+            # a ratio taken for this workload's shape, else one that covers the kernel
+            if fields.get("workload") == workload and ratio is None:
+                ratio = float(fields["traffic_over_algorithmic"])
+            elif "workload" not in fields and generic is None:
+                generic = float(fields["traffic_over_algorithmic"])
+    ratio = ratio if ratio is not None else generic
     return None if ratio is None or algorithmic is None else ratio * algorithmic
 
 
