@@ -312,6 +312,57 @@ moe_status_t moe_ep_pack(const moe_config_t* cfg, int32_t ep_size, const void* x
                          const int32_t* pos, void* x_send, float* w_send, int32_t* e_send,
                          int32_t* send_counts, moe_stream_t stream);
 
+/* The same exchange over peer memory: the rows move by the library's own
+ * stores and loads instead of all-to-alls.  Each rank owns three receive
+ * buffers that every rank can address (peer-mapped device memory over NVLink,
+ * e.g. CUDA IPC or symmetric memory; on one device, plain pointers):
+ * x_recv bf16 [recv_cap, H], w_recv fp32 [recv_cap], y_recv fp32 [recv_cap, H].
+ * A step of rank r:
+ *   1. moe_route and moe_permute on its tokens; moe_ep_expert_counts writes
+ *      counts[e] = rows of its tokens for expert e (int32 [E]);
+ *   2. the caller all-gathers the counts: counts_all int32 [ep_size][E];
+ *   3. moe_ep_plan: the owner's receive buffer is expert-major (its experts in
+ *      order, each expert's rows by source rank, each source's rows in its
+ *      sorted order), so the q-th row of rank r's segment of expert e lands at
+ *      row exp_base[e] + src_base[e] + q of its owner's buffer (int32 [E]
+ *      each); recv_offsets int32 [E/ep_size + 1] are rank r's own segments and
+ *      recv_ident int32 [recv_cap] gets 0, 1, ... for its received rows.  A
+ *      total beyond recv_cap sets a flag in the status word of `ws` (a layer
+ *      workspace; moe_check_device_status reports MOE_ERR_WORKSPACE) and the
+ *      rows beyond it are dropped;
+ *   4. moe_ep_dispatch_peer stores each routed row (H bf16) and its weight into
+ *      the owner's x_recv / w_recv (x_recv, w_recv: device arrays of ep_size
+ *      pointers, index = owner rank);
+ *   5. the caller orders every rank's dispatch before any rank's expert GEMMs
+ *      (a cross-device barrier);
+ *   6. each rank runs its experts as a k = 1 layer over its R received rows
+ *      (R = recv_offsets[E/ep_size]): moe_expert_ffn with T = R, E/ep_size
+ *      experts, offsets = recv_offsets, rows = pos = recv_ident, topk_w =
+ *      w_recv, no shared expert, y = its y_recv (fp32 rows);
+ *   7. a barrier, then moe_shared_expert and moe_ep_combine_peer: out_t = the
+ *      sum over slots j (in order) of the row's output loaded from its owner's
+ *      y_recv (y_recv: a device array of ep_size pointers), rounded to bf16
+ *      first when k > 1, plus the shared expert's row; one bf16 rounding.
+ * The output equals moe_forward's bit for bit.  ep_rank in [0, ep_size).     */
+moe_status_t moe_ep_expert_counts(const moe_config_t* cfg, const int32_t* offsets, int32_t* counts,
+                                  moe_stream_t stream);
+moe_status_t moe_ep_plan(const moe_config_t* cfg, int32_t ep_size, int32_t ep_rank,
+                         const int32_t* counts_all, int32_t* exp_base, int32_t* src_base,
+                         int32_t* recv_offsets, int32_t* recv_ident, int32_t recv_cap, void* ws,
+                         moe_stream_t stream);
+moe_status_t moe_ep_dispatch_peer(const moe_config_t* cfg, int32_t ep_size, int32_t ep_rank,
+                                  const void* x, const int32_t* topk_idx, const float* topk_w,
+                                  const int32_t* offsets, const int32_t* pos,
+                                  const int32_t* exp_base, const int32_t* src_base,
+                                  void* const* x_recv, float* const* w_recv, int32_t recv_cap,
+                                  moe_stream_t stream);
+moe_status_t moe_ep_combine_peer(const moe_config_t* cfg, int32_t ep_size, int32_t ep_rank,
+                                 const int32_t* topk_idx, const int32_t* offsets,
+                                 const int32_t* pos, const int32_t* exp_base,
+                                 const int32_t* src_base, const float* const* y_recv,
+                                 const float* y_shared, void* out, int32_t recv_cap,
+                                 moe_stream_t stream);
+
 /* The shared expert alone (bf16 layers): y_shared fp32 [T, H] =
  * SwiGLU_shared(x) with w13s bf16 [2 Is, H], w2s bf16 [H, Is] (Is =
  * n_shared * I > 0).  ws: moe_workspace_size(cfg) bytes.  Step 6 above; the

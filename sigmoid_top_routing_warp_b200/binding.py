@@ -39,7 +39,8 @@ EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", 
             "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
             "moe_quantize_act", "moe_rmsnorm", "moe_forward_block",
             "moe_backward_workspace_size", "moe_backward", "moe_ep_pack",
-            "moe_shared_expert",
+            "moe_shared_expert", "moe_ep_expert_counts", "moe_ep_plan", "moe_ep_dispatch_peer",
+            "moe_ep_combine_peer",
             "dsa_workspace_size", "dsa_workspace_scores_offset", "dsa_index_scores",
             "dsa_index_topk", "dsa_indexer")
 
@@ -142,6 +143,17 @@ _lib.moe_ep_pack.restype = ctypes.c_int
 _lib.moe_ep_pack.argtypes = [_CFG, ctypes.c_int32] + [_P] * 10
 _lib.moe_shared_expert.restype = ctypes.c_int
 _lib.moe_shared_expert.argtypes = [_CFG] + [_P] * 5 + [ctypes.c_size_t, _P]
+_lib.moe_ep_expert_counts.restype = ctypes.c_int
+_lib.moe_ep_expert_counts.argtypes = [_CFG, _P, _P, _P]
+_lib.moe_ep_plan.restype = ctypes.c_int
+_lib.moe_ep_plan.argtypes = [_CFG, ctypes.c_int32, ctypes.c_int32] + [_P] * 5 + [
+    ctypes.c_int32, _P, _P]
+_lib.moe_ep_dispatch_peer.restype = ctypes.c_int
+_lib.moe_ep_dispatch_peer.argtypes = [_CFG, ctypes.c_int32, ctypes.c_int32] + [_P] * 9 + [
+    ctypes.c_int32, _P]
+_lib.moe_ep_combine_peer.restype = ctypes.c_int
+_lib.moe_ep_combine_peer.argtypes = [_CFG, ctypes.c_int32, ctypes.c_int32] + [_P] * 8 + [
+    ctypes.c_int32, _P]
 _lib.moe_check_device_status.restype = ctypes.c_int
 _lib.moe_check_device_status.argtypes = [_P, _P]
 
@@ -290,6 +302,40 @@ def moe_ep_pack(cfg, ep_size, x, topk_idx, topk_w, offsets, pos, x_send, w_send,
     _check(_lib.moe_ep_pack(ctypes.byref(c), int(ep_size), _ptr(x), _ptr(topk_idx),
                             _ptr(topk_w), _ptr(offsets), _ptr(pos), _ptr(x_send), _ptr(w_send),
                             _ptr(e_send), _ptr(send_counts), _stream(stream)), "moe_ep_pack")
+
+
+def moe_ep_expert_counts(cfg, offsets, counts, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_ep_expert_counts(ctypes.byref(c), _ptr(offsets), _ptr(counts),
+                                     _stream(stream)), "moe_ep_expert_counts")
+
+
+def moe_ep_plan(cfg, ep_size, ep_rank, counts_all, exp_base, src_base, recv_offsets, recv_ident,
+                recv_cap, ws, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_ep_plan(ctypes.byref(c), int(ep_size), int(ep_rank), _ptr(counts_all),
+                            _ptr(exp_base), _ptr(src_base), _ptr(recv_offsets), _ptr(recv_ident),
+                            int(recv_cap), _ptr(ws), _stream(stream)), "moe_ep_plan")
+
+
+def moe_ep_dispatch_peer(cfg, ep_size, ep_rank, x, topk_idx, topk_w, offsets, pos, exp_base,
+                         src_base, x_recv_ptrs, w_recv_ptrs, recv_cap, stream=None):
+    """x_recv_ptrs / w_recv_ptrs: int64 device tensors of the owners' buffer addresses."""
+    c = cfg.c()
+    _check(_lib.moe_ep_dispatch_peer(ctypes.byref(c), int(ep_size), int(ep_rank), _ptr(x),
+                                     _ptr(topk_idx), _ptr(topk_w), _ptr(offsets), _ptr(pos),
+                                     _ptr(exp_base), _ptr(src_base), _ptr(x_recv_ptrs),
+                                     _ptr(w_recv_ptrs), int(recv_cap), _stream(stream)),
+           "moe_ep_dispatch_peer")
+
+
+def moe_ep_combine_peer(cfg, ep_size, ep_rank, topk_idx, offsets, pos, exp_base, src_base,
+                        y_recv_ptrs, y_shared, out, recv_cap, stream=None):
+    c = cfg.c()
+    _check(_lib.moe_ep_combine_peer(ctypes.byref(c), int(ep_size), int(ep_rank), _ptr(topk_idx),
+                                    _ptr(offsets), _ptr(pos), _ptr(exp_base), _ptr(src_base),
+                                    _ptr(y_recv_ptrs), _ptr(y_shared), _ptr(out), int(recv_cap),
+                                    _stream(stream)), "moe_ep_combine_peer")
 
 
 def moe_shared_expert(cfg, x, w13s, w2s, y_shared, ws, stream=None):

@@ -1123,6 +1123,11 @@ moe_status_t moe_check_device_status(void* ws, moe_stream_t stream) {
     MOE_CUDA(cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
     if (words[0] & moe::DEV_STATUS_TIMEOUT)
         return fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (status 0x%x)", words[0]);
+    if (words[0] & moe::DEV_STATUS_CAPACITY)
+        return fail(MOE_ERR_WORKSPACE,
+                    "an expert-parallel receive buffer was smaller than the rows sent to it "
+                    "(status 0x%x): the rows beyond it were dropped",
+                    words[0]);
     if (dirty >= 0)
         return fail(MOE_ERR_WORKSPACE,
                     "tile-claim counter word %d was %d after the stream drained: a launch "

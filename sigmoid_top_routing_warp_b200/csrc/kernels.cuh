@@ -8,7 +8,7 @@
 namespace moe {
 
 // Device status word bits (stored in the workspace).
-enum : int { DEV_STATUS_TIMEOUT = 1 };
+enum : int { DEV_STATUS_TIMEOUT = 1, DEV_STATUS_CAPACITY = 4 };
 
 // The workspace's first 256 bytes: word 0 is the status word; words
 // kSchedFirstWord .. kStatusWords - 1 hold the persistent GEMMs' tile-claim

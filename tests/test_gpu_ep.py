@@ -158,3 +158,62 @@ def test_virtual_ranks_dots3_decode_shape(B, W):
                                           tokens=None if r == 0 else [0, wl.T - 1])
         print("dots3 N=8 rank %d: vs moe_forward rel-L2 %.1e (%.1f%% bit-equal), vs oracle "
               "rel-L2 %.2e max-abs/rms %.2e" % (r, rel, 100 * same, orel, omx))
+
+
+@pytest.mark.parametrize("N", [2, 4, 8])
+def test_peer_exchange_virtual_ranks_small(B, W, N):
+    """The peer-memory form (moe_ep_expert_counts, moe_ep_plan,
+    moe_ep_dispatch_peer, moe_ep_combine_peer) on N virtual ranks: every
+    rank's output equals moe_forward's bit for bit."""
+    from sigmoid_top_routing_warp_b200 import ep
+    wl = W.Workload("ep_peer", T=96, H=512, E=256, k=8, I=128, n_shared=1, seed=19)
+    inp = W.make_inputs(wl, device="cuda")
+    xs = tokens_of(W, wl, N, wl.T, seed=60 + N)
+    cfg = mk_cfg(B, wl, wl.T)
+    outs = ep.ep_forward_peer_virtual(cfg, xs, inp["w_router"], inp["bias"], inp["w13"],
+                                      inp["w2"], inp["w13s"], inp["w2s"])
+    torch.cuda.synchronize()
+    for r in range(N):
+        check_rank(B, cfg, inp, xs[r], outs[r], "peer N=%d rank %d" % (N, r),
+                   tokens=[0, wl.T // 2, wl.T - 1])
+
+
+def test_peer_exchange_dots3_decode_shape(B, W):
+    """The dots3 decode shape over 8 virtual ranks of 32 experts with the
+    peer-memory exchange: bit-identical to moe_forward on every rank."""
+    from sigmoid_top_routing_warp_b200 import ep
+    wl = W.WORKLOADS["decode"]
+    inp = W.make_inputs(wl, device="cuda")
+    N = 8
+    xs = [inp["x"]] + tokens_of(W, wl, N - 1, wl.T, seed=91)
+    cfg = mk_cfg(B, wl, wl.T)
+    outs = ep.ep_forward_peer_virtual(cfg, xs, inp["w_router"], inp["bias"], inp["w13"],
+                                      inp["w2"], inp["w13s"], inp["w2s"])
+    torch.cuda.synchronize()
+    for r in range(N):
+        check_rank(B, cfg, inp, xs[r], outs[r], "peer dots3 rank %d" % r,
+                   tokens=None if r == 0 else [0, wl.T - 1])
+
+
+def test_peer_plan_flags_a_receive_buffer_too_small(B, W):
+    """Rows beyond a rank's receive capacity are dropped and flagged in the
+    status word: moe_check_device_status reports MOE_ERR_WORKSPACE."""
+    wl = W.Workload("ep_cap", T=64, H=512, E=64, k=4, I=128, seed=23)
+    inp = W.make_inputs(wl, device="cuda")
+    cfg = mk_cfg(B, wl, wl.T)
+    ws = B.alloc_workspace(cfg)
+    N, el = 2, 32
+    counts_all = torch.full((N, wl.E), 5, dtype=torch.int32, device="cuda")  # 320 rows per rank
+    eb = torch.empty((wl.E,), dtype=torch.int32, device="cuda")
+    sb = torch.empty_like(eb)
+    ro = torch.empty((el + 1,), dtype=torch.int32, device="cuda")
+    ident = torch.empty((100,), dtype=torch.int32, device="cuda")
+    B.moe_ep_plan(cfg, N, 1, counts_all, eb, sb, ro, ident, 100, ws)
+    with pytest.raises(B.MoeError) as ei:
+        B.moe_check_device_status(ws)
+    assert ei.value.status == B.MOE_ERR_WORKSPACE
+    # the plan itself: expert-major layout, sources in rank order
+    assert (eb.cpu().numpy() == np.tile(np.arange(el) * 10, N)).all()
+    assert (sb.cpu().numpy() == 5).all()
+    assert (ro.cpu().numpy() == np.arange(el + 1) * 10).all()
+    assert (ident.cpu().numpy() == np.arange(100)).all()
