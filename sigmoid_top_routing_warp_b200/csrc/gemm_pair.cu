@@ -19,10 +19,14 @@
 // value (lane r) and the up value (lane r + 8) of one feature, and SwiGLU is
 // computed in registers.
 //
-// Epilogue: tensor memory -> registers -> per-warp shared-memory transpose ->
-// 16-byte global stores of whole token rows (32 or 64 contiguous bytes per
-// warp and row).  Two accumulator buffers (2 x 256 columns) let the epilogue
-// of one tile overlap the main loop of the next.
+// Epilogue: tensor memory -> registers -> global stores.  The gate/up GEMM
+// stores its SwiGLU outputs straight from registers, which frees the shared
+// memory of a seventh operand stage (2.41-2.47 -> 2.34 ms at prefill); the
+// down GEMM, whose output is four times larger, goes through per-warp
+// shared-memory transposes for 16-byte stores of whole token rows (stored
+// straight from registers it took twice as long).  Two accumulator buffers
+// (2 x 256 columns) let the epilogue of one tile overlap the main loop of the
+// next.
 //
 // Gate/up tiles are claimed at run time: the leader's weight producer takes the next
 // tile index from a counter in the workspace status block and posts it to
@@ -50,10 +54,17 @@ constexpr int kPHalf = kPairTokens / 2;            // token rows per CTA
 constexpr int kPWBytes = 128 * kPBK * 2;           // 16 KB of weights per CTA
 constexpr int kPXBytes = kPHalf * kPBK * 2;        // 16 KB of tokens per CTA
 constexpr int kPStage = kPWBytes + kPXBytes;       // 32 KB
-constexpr int kPStages = 6;
-constexpr int kPEpiBytes = 4 * 4096;               // per-warp transpose buffers
 constexpr int kPBarBytes = 256;
-constexpr int kPSmem = 1024 + kPStages * kPStage + kPEpiBytes + kPBarBytes;
+// The gate/up GEMM stores its SwiGLU outputs straight from registers and
+// gives the operand ring a seventh stage; the down GEMM's larger output goes
+// through per-warp shared-memory transposes (16-byte stores), six stages.
+template <int EPI>
+struct PCfg {
+    static constexpr int STAGES = EPI == EPI_SWIGLU ? 7 : 6;
+    static constexpr int EPI_BYTES = EPI == EPI_SWIGLU ? 0 : 4 * 4096;
+    static constexpr int SMEM = 1024 + STAGES * kPStage + EPI_BYTES + kPBarBytes;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
 constexpr int kPTmemCols = 2 * kPairTokens;        // two 256-column accumulators
 constexpr long long kPWaitLimit = 1ll << 31;
 constexpr int kPRing = 4;                          // claimed tile ids in flight
@@ -61,7 +72,6 @@ constexpr int kPSchedWord = 32;                    // first scheduling word in t
 // consumers of a ring slot: both CTAs' two producers and 4 epilogue warps, and
 // the leader's MMA thread
 constexpr int kPRingReaders = 2 * (2 + 4) + 1;
-static_assert(kPSmem <= 232448, "shared memory budget");
 
 struct PTile {
     int prob, exp, row0, nvalid, f0;
@@ -177,8 +187,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
+    constexpr int kPStages = PCfg<EPI>::STAGES;
     uint8_t* epi_buf = smem + kPStages * kPStage;
-    uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + kPEpiBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi_buf + PCfg<EPI>::EPI_BYTES);
     uint64_t* empty = full + kPStages;
     uint64_t* tfull = empty + kPStages;
     uint64_t* tempty = tfull + 2;
@@ -378,9 +389,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
             const uint32_t col0 = buf * kPairTokens;
             if (EPI == EPI_SWIGLU) {
-                // this warp: features fbase .. fbase + 15 (gate lanes 32q + 16h + t/4)
+                // this warp: features fbase .. fbase + 15 (gate lanes 32q + 16h + t/4);
+                // thread t holds feature 8h + t/4 of tokens 8i + 2(t%4) + {0, 1}
                 const int fbase = tl.f0 + 64 * (int)cta + 16 * q;
-                __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stage);  // [32 tokens][16]
                 for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
                     uint32_t r0[16], r1[16];
                     tmem_ld_16x256b_x4(tmem_base + ((uint32_t)(32 * q) << 16) + col0 + c0, r0);
@@ -389,26 +400,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t* r = h ? r1 : r0;
+                        const int f = fbase + 8 * h + (lane >> 2);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const float g = __uint_as_float(r[4 * i + e]);
-                                const float u = __uint_as_float(r[4 * i + 2 + e]);
-                                const int tok = 8 * i + 2 * (lane & 3) + e;
-                                st[tok * 16 + 8 * h + (lane >> 2)] = __float2bfloat16_rn(silu_f(g) * u);
+                                const int tok = c0 + 8 * i + 2 * (lane & 3) + e;
+                                if (tok < tl.nvalid && f < p.n_feat) {
+                                    const float g = __uint_as_float(r[4 * i + e]);
+                                    const float u = __uint_as_float(r[4 * i + 2 + e]);
+                                    out[(size_t)(tl.row0 + tok) * p.ld_out + f] =
+                                        __float2bfloat16_rn(silu_f(g) * u);
+                                }
                             }
                     }
-                    __syncwarp();
-#pragma unroll
-                    for (int it = 0; it < 2; ++it) {
-                        const int tok = 16 * it + (lane >> 1), half = lane & 1;
-                        const int f = fbase + 8 * half;
-                        if (c0 + tok < tl.nvalid && f < p.n_feat)
-                            *reinterpret_cast<uint4*>(out + (size_t)(tl.row0 + c0 + tok) * p.ld_out + f) =
-                                *reinterpret_cast<const uint4*>(st + tok * 16 + 8 * half);
-                    }
-                    __syncwarp();
                 }
             } else {
                 // this warp: features fbase .. fbase + 31 (lane = feature)
@@ -484,6 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 
 template <int EPI>
 static cudaError_t launch_pair_t(const PairParams& params, int grid, cudaStream_t s) {
+    constexpr int kPSmem = PCfg<EPI>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(pair_gemm_kernel<EPI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
     if (e != cudaSuccess) return e;

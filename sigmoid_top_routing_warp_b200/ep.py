@@ -276,7 +276,9 @@ class PeerBuffers:
     ranks' addresses.  recv_cap rows: T * k * ep_size covers any routing."""
 
     def __init__(self, cfg, ep_size, group=None, device=None):
+        import torch.distributed as dist
         import torch.distributed._symmetric_memory as symm
+        group = group if group is not None else dist.group.WORLD
         dev = device or torch.device("cuda", torch.cuda.current_device())
         self.cap = cfg.T * cfg.k * ep_size
         shapes = {"x": ((self.cap, cfg.H), torch.bfloat16), "w": ((self.cap,), torch.float32),
@@ -284,7 +286,7 @@ class PeerBuffers:
         self.local, self.ptrs, self._handles = {}, {}, []
         for key, (shape, dt) in shapes.items():
             t = symm.empty(*shape, dtype=dt, device=dev)
-            h = symm.rendezvous(t, group if group is not None else "0")
+            h = symm.rendezvous(t, group)
             self.local[key] = t
             self._handles.append(h)
             self.ptrs[key] = torch.tensor([h.get_buffer(r, shape, dt).data_ptr()
