@@ -1181,4 +1181,26 @@ moe_status_t api_make_map_3d_bf16(CUtensorMap* m, const void* ptr, uint64_t d0, 
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
     return MOE_OK;
 }
+
+// Store map of an fp32 or bf16 3-D tensor {d0, d1, d2} (d0 contiguous; byte
+// strides of d1 and d2), box {b0, b1, 1}, no swizzle: a staged row-major
+// [b1][b0] tile in shared memory goes out in one bulk tensor store, clipped
+// at the tensor's edges.
+moe_status_t api_make_map_store_3d(CUtensorMap* m, const void* ptr, int f32, uint64_t d0,
+                                   uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2,
+                                   uint32_t b0, uint32_t b1, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!aligned16(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", what);
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (%d)", what, (int)r);
+    return MOE_OK;
+}
 }  // namespace moe

@@ -36,6 +36,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 namespace moe {
@@ -48,6 +49,9 @@ moe_status_t api_make_map_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t rows
 moe_status_t api_make_map_3d_bf16(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1,
                                   uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
                                   uint32_t b1, uint32_t b2, const char* what);
+moe_status_t api_make_map_store_3d(CUtensorMap* m, const void* ptr, int f32, uint64_t d0,
+                                   uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2,
+                                   uint32_t b0, uint32_t b1, const char* what);
 }  // namespace moe
 
 namespace {
@@ -59,7 +63,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace of moe_backward (256-byte aligned regions).
 struct BLayout {
-    size_t status, offsets, rows, pos, chunk, pstart, tstart, prow, wpad, xpad, dypad, gu, dgu, aw,
+    size_t status, offsets, rows, pos, chunk, pstart, tstart, ttab, prow, wpad, xpad, dypad, gu, dgu, aw,
         dwpart, dxpad, gus, dgus, as, dxsh, dxr, dl, total;
     size_t rmax;  // rows of the padded buffers
 };
@@ -84,6 +88,7 @@ BLayout blayout(const moe_config_t* c) {
     L.chunk = take((size_t)moe::permute_chunks((int)n) * E * 4);
     L.pstart = take((E + 1) * 4);
     L.tstart = take((E + 1) * 4);
+    L.ttab = take((L.rmax / kRowTile + E) * 4);
     L.prow = take(n * 4);
     L.wpad = take(L.rmax * 4);
     L.xpad = take(L.rmax * H * 2);
@@ -137,6 +142,7 @@ struct PlanArgs {
     const int32_t* offsets;
     int32_t* pstart;  // [E + 1] padded segment starts
     int32_t* tstart;  // [E + 1] prefix of 256-row tiles over the padded segments
+    int32_t* ttab;    // [tstart[E]] the expert of each row tile
     int E;
 };
 
@@ -169,6 +175,8 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(const PlanArgs a) {
         a.pstart[a.E] = sp[e];
         a.tstart[a.E] = st[e];
     }
+    // the expert of each row tile
+    for (int r = 0; r < nt; ++r) a.ttab[st[e] - nt + r] = e;
 }
 
 struct BGatherArgs {
@@ -353,12 +361,9 @@ moe_status_t need16(const void* p, const char* name) {
 
 using moe::api_make_map_2d_bf16;
 
-// K-major operand maps: [rows, cols] bf16, box {64, 128} (A) or {64, 256} (B).
+// K-major operand maps: [rows, cols] bf16, box {64, 128}.
 moe_status_t kmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
     return api_make_map_2d_bf16(m, p, rows, cols, 64, 128, what);
-}
-moe_status_t kmapB(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
-    return api_make_map_2d_bf16(m, p, rows, cols, 64, 256, what);
 }
 // MN-major operand map of a row-major [K rows, MN cols] bf16 matrix: the 3-D
 // view {64, rows, MN / 64} (strides: a row, 64 elements), box {64, 64, 2}:
@@ -366,11 +371,6 @@ moe_status_t kmapB(CUtensorMap* m, const void* p, size_t rows, size_t cols, cons
 // chunks.  MN is a multiple of 64 for every operand here.
 moe_status_t mnmap(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
     return moe::api_make_map_3d_bf16(m, p, 64, rows, (cols + 63) / 64, cols * 2, 128, 64, 64, 2,
-                                     what);
-}
-// The same for a B operand: box {64, 64, 4}, 256 consecutive MN elements.
-moe_status_t mnmapB(CUtensorMap* m, const void* p, size_t rows, size_t cols, const char* what) {
-    return moe::api_make_map_3d_bf16(m, p, 64, rows, (cols + 63) / 64, cols * 2, 128, 64, 64, 4,
                                      what);
 }
 
@@ -438,6 +438,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
     int32_t* pos = at<int32_t>(ws, L.pos);
     int32_t* pstart = at<int32_t>(ws, L.pstart);
     int32_t* tstart = at<int32_t>(ws, L.tstart);
+    int32_t* ttab = at<int32_t>(ws, L.ttab);
     int32_t* prow = at<int32_t>(ws, L.prow);
     float* wpad = at<float>(ws, L.wpad);
     uint16_t* xpad = at<uint16_t>(ws, L.xpad);
@@ -457,6 +458,32 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
     const int ld_dl = (int)align_up(E, 64);
     int sms = 0;
     BW_TRY(moe::api_sm_count(&sms));
+    // K-major B maps: boxes of 128 rows and of 16, 32 and 64 rows for the
+    // ragged row tiles
+    auto kB = [&](moe::BwdProblem& q, const void* ptr, size_t r, size_t c, const char* w) {
+        for (int i = 0; i < 3; ++i) BW_TRY(api_make_map_2d_bf16(&q.tbs[i], ptr, r, c, 64, 16u << i, w));
+        return kmap(&q.tb, ptr, r, c, w);
+    };
+    // Launch one backward GEMM; a store epilogue first gets the store map of
+    // each problem's output: 16-row boxes over padded segments (whose row
+    // tiles end on a multiple of 16), 32-row boxes elsewhere.
+    auto gemm = [&](int epi, moe::BwdParams& P, const char* what) -> moe_status_t {
+        if (epi == moe::BEPI_STORE)
+            for (int i = 0; i < P.n_problems; ++i) {
+                moe::BwdProblem& p = P.p[i];
+                const size_t rows = p.rows_as_k ? (size_t)p.N : p.seg ? R : (size_t)p.n_rows;
+                const size_t groups = p.rows_as_k ? (size_t)p.n_grp : 1;
+                const size_t es = p.out_f32 ? 4 : 2;
+                const size_t gstride = groups > 1 ? (size_t)p.out_grp * es : rows * p.ld_out * es;
+                BW_TRY(moe::api_make_map_store_3d(&p.to, p.out, p.out_f32, p.M, rows, groups,
+                                                  (size_t)p.ld_out * es, gstride, 32,
+                                                  (p.rows_as_k || !p.seg) ? 32 : 16,
+                                                  "gradient output"));
+            }
+        P.status = status;
+        BW_CUDA(moe::launch_bwd_gemm(epi, P, sms, s), what);
+        return MOE_OK;
+    };
     cudaEvent_t ev[MOE_NUM_BWD_STAGES + 1] = {};
     if (stage_events)
         for (int i = 0; i <= MOE_NUM_BWD_STAGES; ++i) ev[i] = static_cast<cudaEvent_t>(stage_events[i]);
@@ -478,7 +505,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
     pa.E = E;
     BW_CUDA(moe::launch_permute(pa, s), "permute launch");
     // 2. padded segments
-    PlanArgs pl{offsets, pstart, tstart, E};
+    PlanArgs pl{offsets, pstart, tstart, ttab, E};
     bwd_plan_kernel<<<1, 1024, 0, s>>>(pl);
     BW_CUDA(cudaGetLastError(), "plan launch");
     // 3. gather
@@ -494,10 +521,10 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         memset(&P, 0, sizeof(P));
         moe::BwdProblem& p = P.p[0];
         BW_TRY(kmap(&p.ta, w13, (size_t)E * 2 * I, H, "w13"));
-        BW_TRY(kmapB(&p.tb, xpad, R, H, "padded x"));
-        BW_TRY(kmap(&p.tb_half, xpad, R, H, "padded x"));
+        BW_TRY(kB(p, xpad, R, H, "padded x"));
         p.seg = pstart;
         p.tstart = tstart;
+        p.ttab = ttab;
         p.n_grp = E;
         p.M = 2 * I;
         p.K = H;
@@ -509,8 +536,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[1];
             BW_TRY(kmap(&q.ta, w13s, (size_t)2 * Is, H, "w13s"));
-            BW_TRY(kmapB(&q.tb, x, T, H, "x"));
-            BW_TRY(kmap(&q.tb_half, x, T, H, "x"));
+            BW_TRY(kB(q, x, T, H, "x"));
             q.n_grp = 1;
             q.n_rows = T;
             q.M = 2 * Is;
@@ -520,8 +546,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
             q.out_f32 = 1;
             P.n_problems = 2;
         }
-        P.status = status;
-        BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "gate/up recompute GEMM launch");
+        BW_TRY(gemm(moe::BEPI_STORE, P, "gate/up recompute GEMM launch"));
     }
     BW_TRY(mark(2));
     // 5. dA' = dY W2_e with the SwiGLU backward in the epilogue
@@ -530,11 +555,11 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         memset(&P, 0, sizeof(P));
         moe::BwdProblem& p = P.p[0];
         BW_TRY(mnmap(&p.ta, w2, (size_t)E * H, I, "w2"));
-        BW_TRY(kmapB(&p.tb, dypad, R, H, "padded dout"));
-        BW_TRY(kmap(&p.tb_half, dypad, R, H, "padded dout"));
+        BW_TRY(kB(p, dypad, R, H, "padded dout"));
         p.a_mn = 1;
         p.seg = pstart;
         p.tstart = tstart;
+        p.ttab = ttab;
         p.n_grp = E;
         p.M = I;
         p.K = H;
@@ -553,8 +578,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[1];
             BW_TRY(mnmap(&q.ta, w2s, H, Is, "w2s"));
-            BW_TRY(kmapB(&q.tb, dout, T, H, "dout"));
-            BW_TRY(kmap(&q.tb_half, dout, T, H, "dout"));
+            BW_TRY(kB(q, dout, T, H, "dout"));
             q.a_mn = 1;
             q.n_grp = 1;
             q.n_rows = T;
@@ -569,8 +593,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
             q.ld_aw = Is;
             P.n_problems = 2;
         }
-        P.status = status;
-        BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_DSWIGLU, P, sms, s), "down backward GEMM launch");
+        BW_TRY(gemm(moe::BEPI_DSWIGLU, P, "down backward GEMM launch"));
     }
     BW_TRY(mark(3));
     // 6. router gradient
@@ -588,11 +611,11 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         int np = 0;
         moe::BwdProblem& p = P.p[np++];
         BW_TRY(mnmap(&p.ta, w13, (size_t)E * 2 * I, H, "w13"));
-        BW_TRY(kmapB(&p.tb, dgu, R, 2 * I, "padded dgate/dup"));
-        BW_TRY(kmap(&p.tb_half, dgu, R, 2 * I, "padded dgate/dup"));
+        BW_TRY(kB(p, dgu, R, 2 * I, "padded dgate/dup"));
         p.a_mn = 1;
         p.seg = pstart;
         p.tstart = tstart;
+        p.ttab = ttab;
         p.n_grp = E;
         p.M = H;
         p.K = 2 * I;
@@ -602,8 +625,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& q = P.p[np++];
             BW_TRY(mnmap(&q.ta, w13s, (size_t)2 * Is, H, "w13s"));
-            BW_TRY(kmapB(&q.tb, dgus, T, 2 * Is, "shared dgate/dup"));
-            BW_TRY(kmap(&q.tb_half, dgus, T, 2 * Is, "shared dgate/dup"));
+            BW_TRY(kB(q, dgus, T, 2 * Is, "shared dgate/dup"));
             q.a_mn = 1;
             q.n_grp = 1;
             q.n_rows = T;
@@ -615,8 +637,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         }
         moe::BwdProblem& r = P.p[np++];
         BW_TRY(mnmap(&r.ta, w_router, E, H, "w_router"));
-        BW_TRY(kmapB(&r.tb, dl, T, ld_dl, "router dlogits"));
-        BW_TRY(kmap(&r.tb_half, dl, T, ld_dl, "router dlogits"));
+        BW_TRY(kB(r, dl, T, ld_dl, "router dlogits"));
         r.a_mn = 1;
         r.n_grp = 1;
         r.n_rows = T;
@@ -626,8 +647,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         r.ld_out = H;
         r.out_f32 = 1;
         P.n_problems = np;
-        P.status = status;
-        BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "input gradient GEMM launch");
+        BW_TRY(gemm(moe::BEPI_STORE, P, "input gradient GEMM launch"));
     }
     BW_TRY(mark(5));
     // 8. weight gradients: K = the expert's padded rows (or the T tokens)
@@ -637,7 +657,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         int np = 0;
         moe::BwdProblem& p = P.p[np++];  // dW2_e[h][i] = sum_r dY[r][h] (w a)[r][i]
         BW_TRY(mnmap(&p.ta, aw, R, I, "padded w*a"));
-        BW_TRY(mnmapB(&p.tb, dypad, R, H, "padded dout"));
+        BW_TRY(mnmap(&p.tb, dypad, R, H, "padded dout"));
         p.a_mn = p.b_mn = 1;
         p.rows_as_k = 1;
         p.seg = pstart;
@@ -650,7 +670,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         p.out_f32 = 1;
         moe::BwdProblem& q = P.p[np++];  // dW13_e[j][h] = sum_r dGU[r][j] X[r][h]
         BW_TRY(mnmap(&q.ta, xpad, R, H, "padded x"));
-        BW_TRY(mnmapB(&q.tb, dgu, R, 2 * I, "padded dgate/dup"));
+        BW_TRY(mnmap(&q.tb, dgu, R, 2 * I, "padded dgate/dup"));
         q.a_mn = q.b_mn = 1;
         q.rows_as_k = 1;
         q.seg = pstart;
@@ -664,7 +684,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         if (Is > 0) {
             moe::BwdProblem& a2 = P.p[np++];  // dW2s[h][i]
             BW_TRY(mnmap(&a2.ta, as, T, Is, "shared a"));
-            BW_TRY(mnmapB(&a2.tb, dout, T, H, "dout"));
+            BW_TRY(mnmap(&a2.tb, dout, T, H, "dout"));
             a2.a_mn = a2.b_mn = 1;
             a2.rows_as_k = 1;
             a2.n_grp = 1;
@@ -676,7 +696,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
             a2.out_f32 = 1;
             moe::BwdProblem& a3 = P.p[np++];  // dW13s[j][h]
             BW_TRY(mnmap(&a3.ta, x, T, H, "x"));
-            BW_TRY(mnmapB(&a3.tb, dgus, T, 2 * Is, "shared dgate/dup"));
+            BW_TRY(mnmap(&a3.tb, dgus, T, 2 * Is, "shared dgate/dup"));
             a3.a_mn = a3.b_mn = 1;
             a3.rows_as_k = 1;
             a3.n_grp = 1;
@@ -689,7 +709,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         }
         moe::BwdProblem& g = P.p[np++];  // dW_g[e][h] = sum_t dL[t][e] x[t][h]
         BW_TRY(mnmap(&g.ta, x, T, H, "x"));
-        BW_TRY(mnmapB(&g.tb, dl, T, ld_dl, "router dlogits"));
+        BW_TRY(mnmap(&g.tb, dl, T, ld_dl, "router dlogits"));
         g.a_mn = g.b_mn = 1;
         g.rows_as_k = 1;
         g.n_grp = 1;
@@ -700,8 +720,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
         g.ld_out = H;
         g.out_f32 = 1;
         P.n_problems = np;
-        P.status = status;
-        BW_CUDA(moe::launch_bwd_gemm(moe::BEPI_STORE, P, sms, s), "weight gradient GEMM launch");
+        BW_TRY(gemm(moe::BEPI_STORE, P, "weight gradient GEMM launch"));
     }
     BW_TRY(mark(6));
     // 9. dx

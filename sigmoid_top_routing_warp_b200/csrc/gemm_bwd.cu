@@ -1,48 +1,33 @@
-// gemm_bwd.cu -- the grouped GEMMs of the layer's backward pass on the
-// 5th-generation tensor cores (tcgen05 + tensor memory), fed by TMA.
+// gemm_bwd.cu -- the grouped GEMMs of the layer's backward pass on CTA pairs
+// (tcgen05 cta_group::2): K- or MN-major operands, token rows along N or K
+// over an expert's row segment, a 256 x 256 tile over two SMs.
 //
-// The backward pass is the chain rule through the forward pass that
-// "Xiaohongshu dots3 note Open Source Deep Dive" describes (§3.1: gate ->
-// scores -> top-k -> renormalise -> shared + weighted routed sum; §8.2:
-// gmm1 -> swiglu -> gmm2), with the expert choice held fixed.  Its GEMMs
-// contract along three different axes:
-//   - recomputed gate/up pre-activations  G|U = X W13^T        (K = hidden)
-//   - the down projection's input grad    dA  = dY W2_e        (K = hidden,
-//                                           W2_e read with I contiguous)
-//   - the input grad                      dX  = dG|dU W13_e    (K = 2I,
-//                                           W13_e read with H contiguous)
-//   - the weight grads                    dW2_e = dY_e^T (w A)_e,
-//                                          dW13_e = dG|dU_e^T X_e
-//                                           (K = the expert's token rows)
-// so, unlike the forward kernels, operands come K-major or MN-major (the
-// tensor core reads either from shared memory; the instruction descriptor
-// says which), and K may run over an expert's row segment.
+// Source of the operation: the chain rule through the forward pass of
+// "Xiaohongshu dots3 note Open Source Deep Dive" §3.1 / §8.2 (see
+// backward.cu), the expert choice held fixed.
 //
-// Tile: 128 x 256 (M = output features in tensor-memory lanes, N = token
-// rows or output columns), K step 64; the MMA's N is the tile's valid
-// columns rounded up to 16.  Roles (352 threads, one CTA per SM,
-// persistent, static round-robin over the tile list):
-//   warp 0      TMA producer of the A operand (one 16 KB box per stage: K-major
-//               {64, 128}, or MN-major {64, 64, 2} of a 3-D view that brings
-//               two 64-wide chunks), warp 10 of the B operand (32 KB: {64, 256}
-//               or {64, 64, 4}); two issuing threads, because one thread's
-//               tensor copies top out well below the SM's L2 bandwidth
-//   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2..9  epilogue (tcgen05.ld 32x32b: lane = feature m): two warps per
-//               tensor-memory lane quadrant, each taking half of the tile's
-//               columns; stores go through a per-warp shared-memory transpose
-//               so that each thread writes 16 bytes of one output row
-// Two 256-column accumulators (all of tensor memory) let the epilogue of one
-// tile overlap the main loop of the next.  Row segments are padded to 16 rows by the caller, so a
-// segment ends on an MMA boundary: a K step whose 64 rows run past the
-// segment issues only the MMAs inside it.
+// Why pairs.  A CTA of the pair stages its own 128 rows of A and half of the
+// tile's N columns of B: 32 KB per 64-deep K step for 2 M MACs, where a
+// single-CTA 128 x 256 tile needs 48 KB for the same work, and five or six
+// stages fit in shared memory instead of four.  The leader issues one
+// M = 256 MMA per 16-deep K slice; its commits arrive on both CTAs' barriers.
+// D[m, n] sits in the tensor memory of the CTA that owns row m: each CTA's
+// epilogue writes its 128 rows.
 //
-// Every mbarrier wait is bounded (see wait_bar): on timeout the CTA records
-// DEV_STATUS_TIMEOUT, stops, waits for its copies and MMAs in flight
-// (bounded), frees tensor memory and returns.
+// N per tile: token rows (K-major B) use the tile's valid rows rounded up to
+// 16, each CTA supplying half of them; output columns (MN-major B) use 256.
+//
+// Roles per CTA (352 threads): warp 0 loads A and (leader) sets the stage's
+// expected bytes for both CTAs, warp 1 loads B, warp 2 holds the tensor
+// memory and (leader, one thread) issues the MMAs, warps 3..10 are the
+// epilogue (two per lane quadrant, half the columns each; staged tiles leave
+// in bulk tensor stores, or the SwiGLU backward in registers).  Static
+// round-robin of tiles over pairs.
+// Every wait is bounded; on timeout a CTA records DEV_STATUS_TIMEOUT, stops,
+// drains what it issued, meets its peer at the last cluster barrier and
+// frees its tensor memory.
 #include "kernels.cuh"
 #include "ptx.cuh"
-#include "tiles.cuh"
 
 #include <cuda_bf16.h>
 
@@ -50,143 +35,183 @@ namespace moe {
 
 namespace {
 
-constexpr int kBEpiWarps = 8;
-constexpr int kBThreads = 32 * (3 + kBEpiWarps);
-constexpr int kBProdB = 2 + kBEpiWarps;           // producer warp of the B operand
-constexpr int kBBK = 64;                          // K per stage
-constexpr int kBT = 128;                          // tile M (tensor-memory lanes)
-constexpr int kBN = 256;                          // tile N (columns)
-constexpr int kBABytes = kBT * kBBK * 2;          // 16 KB of A per stage
-constexpr int kBBBytes = kBN * kBBK * 2;          // 32 KB of B per stage
-constexpr int kBStage = kBABytes + kBBBytes;
-constexpr int kBStages = 4;
-constexpr uint32_t kBChunk = kBBK * 128;          // one 64-wide MN chunk: 64 K rows x 128 B
-constexpr int kBBarBytes = 256;
-constexpr int kBEpiBytes = kBEpiWarps * 32 * 32 * 4;  // per-warp [32 columns][32 features] fp32
-constexpr int kBSmem = 1024 + kBStages * kBStage + kBEpiBytes + kBBarBytes;
-constexpr int kBTmemCols = 2 * kBN;
-static_assert(kBSmem <= 232448, "shared memory budget");
+constexpr int kQEpiWarps = 8;
+constexpr int kQThreads = 32 * (3 + kQEpiWarps);
+constexpr int kQMmaWarp = 2;                       // warps 0, 1 load; 2 issues; 3..10 drain
+constexpr int kQEpi0 = kQMmaWarp + 1;
+constexpr int kQBK = 64;
+constexpr int kQM = 256;                           // pair tile M (128 rows per CTA)
+constexpr int kQN = 256;                           // tile N (128 per CTA staged)
+constexpr int kQOpBytes = 128 * kQBK * 2;          // 16 KB: A or the CTA's half of B
+constexpr int kQStage = 2 * kQOpBytes;
+constexpr uint32_t kQChunk = kQBK * 128;           // one 64-wide MN chunk: 64 K rows x 128 B
+constexpr int kQBarBytes = 256;
+constexpr int kQTmemCols = 2 * kQN;
+constexpr long long kQWaitLimit = 1ll << 31;
+// Shared memory per epilogue: stores keep five operand stages and two 4 KB
+// staging tiles per epilogue warp; the SwiGLU backward needs no staging and
+// takes six stages.
+template <int EPI>
+struct QCfg {
+    static constexpr int STAGES = EPI == BEPI_DSWIGLU ? 6 : 5;
+    static constexpr int SBUF = EPI == BEPI_DSWIGLU ? 0 : 2;
+    static constexpr int EPI_BYTES = kQEpiWarps * SBUF * 4096;
+    static constexpr int SMEM = 1024 + STAGES * kQStage + EPI_BYTES + kQBarBytes;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
 
-struct BTile {
+struct QTile {
     int prob, grp, m0, n0, nvalid, k0, k1;
 };
 
-__device__ __forceinline__ int bprob_tiles(const BwdProblem& p) {
-    const int mt = (p.M + kBT - 1) / kBT;
-    if (p.rows_as_k) return p.n_grp * mt * ((p.N + kBN - 1) / kBN);
-    if (p.seg == nullptr) return mt * ((p.n_rows + kBN - 1) / kBN);
+__device__ __forceinline__ int qprob_tiles(const BwdProblem& p) {
+    const int mt = (p.M + kQM - 1) / kQM;
+    if (p.rows_as_k) return p.n_grp * mt * ((p.N + kQN - 1) / kQN);
+    if (p.seg == nullptr) return mt * ((p.n_rows + kQN - 1) / kQN);
     return mt * __ldg(p.tstart + p.n_grp);
 }
 
-__device__ __forceinline__ int btotal(const BwdParams& P) {
+__device__ __forceinline__ int qtotal(const BwdParams& P) {
     int n = 0;
-    for (int i = 0; i < P.n_problems; ++i) n += bprob_tiles(P.p[i]);
+    for (int i = 0; i < P.n_problems; ++i) n += qprob_tiles(P.p[i]);
     return n;
 }
 
-// Tile t of the launch.  Order inside a problem: group, feature tile, then
-// row (or column) tile, so that CTAs working at once share operand tiles in L2.
-__device__ __forceinline__ bool btile_at(const BwdParams& P, int t, BTile& o) {
+// Tile t: group, N tile, then M tile innermost.  With token rows along N the
+// pairs running together share a tile of token rows while the group's
+// weights (at most a few tens of MB) stay in L2 across its row tiles.  With
+// rows as K (weight gradients, out[n][m], m contiguous) the pairs running
+// together write adjacent column ranges of the same output rows, so the
+// fp32 gradients reach DRAM as runs of whole rows rather than 1 KB pieces.
+__device__ __forceinline__ void qtile_at(const BwdParams& P, int t, QTile& o) {
     for (int pi = 0; pi < P.n_problems; ++pi) {
         const BwdProblem& p = P.p[pi];
-        const int n = bprob_tiles(p);
+        const int n = qprob_tiles(p);
         if (t >= n) {
             t -= n;
             continue;
         }
-        const int mt = (p.M + kBT - 1) / kBT;
+        const int mt = (p.M + kQM - 1) / kQM;
         o.prob = pi;
         if (p.rows_as_k) {
-            const int nt = (p.N + kBN - 1) / kBN;
+            const int nt = (p.N + kQN - 1) / kQN;
             const int g = t / (mt * nt);
             const int l = t - g * mt * nt;
             o.grp = g;
-            o.m0 = (l / nt) * kBT;
-            o.n0 = (l % nt) * kBN;
-            o.nvalid = min(kBN, p.N - o.n0);
+            o.m0 = (l % mt) * kQM;
+            o.n0 = (l / mt) * kQN;
+            o.nvalid = min(kQN, p.N - o.n0);
             o.k0 = p.seg ? __ldg(p.seg + g) : 0;
             o.k1 = p.seg ? __ldg(p.seg + g + 1) : p.n_rows;
         } else if (p.seg == nullptr) {
-            const int nt = (p.n_rows + kBN - 1) / kBN;
             o.grp = 0;
-            o.m0 = (t / nt) * kBT;
-            o.n0 = (t % nt) * kBN;
-            o.nvalid = min(kBN, p.n_rows - o.n0);
+            o.m0 = (t % mt) * kQM;
+            o.n0 = (t / mt) * kQN;
+            o.nvalid = min(kQN, p.n_rows - o.n0);
             o.k0 = 0;
             o.k1 = p.K;
         } else {
-            // largest group g with mt * tstart[g] <= t (a group with no rows has no tiles)
-            int lo = 0, hi = p.n_grp - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (mt * __ldg(p.tstart + mid) <= t) lo = mid; else hi = mid - 1;
+            int g;
+            if (p.ttab != nullptr) {
+                g = __ldg(p.ttab + t / mt);
+            } else {
+                int lo = 0, hi = p.n_grp - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (mt * __ldg(p.tstart + mid) <= t) lo = mid; else hi = mid - 1;
+                }
+                g = lo;
             }
-            const int g = lo;
             const int l = t - mt * __ldg(p.tstart + g);
-            const int ntg = __ldg(p.tstart + g + 1) - __ldg(p.tstart + g);
             o.grp = g;
-            o.m0 = (l / ntg) * kBT;
-            o.n0 = __ldg(p.seg + g) + (l % ntg) * kBN;
-            o.nvalid = min(kBN, __ldg(p.seg + g + 1) - o.n0);
+            o.m0 = (l % mt) * kQM;
+            o.n0 = __ldg(p.seg + g) + (l / mt) * kQN;
+            o.nvalid = min(kQN, __ldg(p.seg + g + 1) - o.n0);
             o.k0 = 0;
             o.k1 = p.K;
         }
-        return true;
+        return;
     }
-    return false;
 }
 
-__device__ __forceinline__ int bk_blocks(const BTile& t) {
-    return t.k1 > t.k0 ? (t.k1 - t.k0 + kBBK - 1) / kBBK : 0;
+__device__ __forceinline__ int qk_blocks(const QTile& t) {
+    return t.k1 > t.k0 ? (t.k1 - t.k0 + kQBK - 1) / kQBK : 0;
 }
 
-// One operand of one stage: a K-major box {64 K, 128 rows} at (k, row0 + mn0)
-// of a 2-D map, or an MN-major box {64, 64 K, 2 chunks} at (0, row0 + k,
-// mn0 / 64) of the 3-D view {64, rows, MN / 64} (chunk c lands kBChunk bytes
-// after chunk c - 1).
-__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* m, int mn_major,
-                                             int mn0, int k, int row0, uint64_t* bar) {
+// MMA N of a tile: token rows (K-major B) trimmed to the valid rows rounded
+// up to 16; output columns (MN-major B, whose halves must start on a 64-wide
+// chunk) the full 256.
+__device__ __forceinline__ int qtile_n(const BwdProblem& p, const QTile& t) {
+    return p.b_mn ? kQN : min(kQN, (t.nvalid + 15) & ~15);
+}
+
+__device__ __forceinline__ bool qwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                      int* status, bool drain = false) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (!drain && *abort_flag) return false;
+        if (clock64() - t0 > kQWaitLimit) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, DEV_STATUS_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// One operand half of one stage into this CTA's shared memory, counted on
+// the leader's barrier: K-major box {64 K, 128 rows} at (k, row0 + mn0), or
+// MN-major box {64, 64 K, 2 chunks} at (0, row0 + k, mn0 / 64).
+__device__ __forceinline__ void qload(uint8_t* dst, const CUtensorMap* m, int mn_major, int mn0,
+                                      int k, int row0, uint32_t bar_cluster) {
     if (!mn_major)
-        tma_load_2d(dst, m, bar, k, row0 + mn0);
+        tma_load_2d_pair(dst, m, bar_cluster, k, row0 + mn0);
     else
-        tma_load_3d(dst, m, bar, 0, row0 + k, mn0 >> 6);
+        tma_load_3d_pair(dst, m, bar_cluster, 0, row0 + k, mn0 >> 6);
 }
 
-// Descriptor of the 16-deep K slice kk of an operand stage.
-__device__ __forceinline__ uint64_t op_desc(uint32_t base, int mn_major, int kk) {
-    return mn_major ? smem_desc_mn_sw128(base + kk * 16 * 128, kBChunk, 1024)
+__device__ __forceinline__ uint64_t qdesc(uint32_t base, int mn_major, int kk) {
+    return mn_major ? smem_desc_mn_sw128(base + kk * 16 * 128, kQChunk, 1024)
                     : smem_desc_k_sw128(base + kk * 32);
 }
 
-__device__ __forceinline__ uint16_t f2bf(float v) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
+__device__ __forceinline__ uint16_t qbf(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
 }  // namespace
 
 template <int EPI>
-__global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdParams P) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kQThreads, 1)
+    bwd_pair_gemm_kernel(const __grid_constant__ BwdParams P) {
+    using C = QCfg<EPI>;
+    constexpr int kQStages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    float* epi_smem = reinterpret_cast<float*>(smem + kBStages * kBStage);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBStages * kBStage + kBEpiBytes);
-    uint64_t* empty = full + kBStages;
-    uint64_t* tfull = empty + kBStages;
+    float* epi_smem = reinterpret_cast<float*>(smem + kQStages * kQStage);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kQStage + C::EPI_BYTES);
+    uint64_t* empty = full + kQStages;
+    uint64_t* tfull = empty + kQStages;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t cta = cluster_ctarank();
+    const bool leader = cta == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kBStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(&full[s], 1);    // the leader's A producer (expected bytes of both CTAs)
+            mbar_init(&empty[s], 1);   // one multicast commit per phase
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kBEpiWarps);
+            mbar_init(&tfull[b], 1);                 // one multicast commit per tile
+            mbar_init(&tempty[b], 2 * kQEpiWarps);   // both CTAs' epilogue warps (leader's copy)
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -196,133 +221,138 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
         for (int pi = 0; pi < P.n_problems; ++pi) {
             tma_prefetch_desc(&P.p[pi].ta);
             tma_prefetch_desc(&P.p[pi].tb);
-            if (!P.p[pi].rows_as_k && !P.p[pi].b_mn) tma_prefetch_desc(&P.p[pi].tb_half);
         }
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_holder, kBTmemCols);
-        tmem_relinquish();
+    if (warp == kQMmaWarp) {
+        tmem_alloc_pair(tmem_holder, kQTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    const int ntiles = btotal(P);
+    const int ntiles = qtotal(P);
 
-    if (warp == 0 || warp == kBProdB) {
-        // ------------------------------------------------ TMA producers
-        // Warp 0 loads A and sets the stage's expected bytes (both operands);
-        // warp kBProdB loads B.  A copy that lands before the expectation is
-        // set leaves the barrier's phase open: warp 0's arrival is pending.
+    if (warp < kQMmaWarp) {
+        // ------------------------------------------------ TMA producers (both CTAs)
         if (lane == 0) {
             const bool pa = warp == 0;
-            int s = 0;
-            uint32_t ph = 0, issued = 0, last_ph = 0;
+            const uint32_t full_leader = mapa_shared(smem_addr(&full[0]), 0);
+            uint32_t it = 0;  // k-blocks of this CTA so far
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-                BTile tl;
-                btile_at(P, t, tl);
+            for (int t = pair; ok && t < ntiles; t += npairs) {
+                QTile tl;
+                qtile_at(P, t, tl);
                 const BwdProblem& p = P.p[tl.prob];
-                const int nkb = bk_blocks(tl);
+                const int nkb = qk_blocks(tl);
                 const int arow = p.rows_as_k ? 0 : tl.grp * p.a_grp_rows;
-                // a row tile with at most 128 valid rows loads a 128-row B box
-                const bool bhalf = !p.rows_as_k && !p.b_mn && tl.nvalid <= kBN / 2;
-                const uint32_t stage_bytes = kBABytes + (bhalf ? kBBBytes / 2 : kBBBytes);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!wait_bar(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
-                    uint8_t* st = smem + s * kBStage;
-                    const int k = tl.k0 + kb * kBBK;
+                const int half = qtile_n(p, tl) >> 1;  // B columns each CTA supplies
+                // K-major B: the smallest box of 16 << b rows that holds them
+                int box = 3;
+                if (!p.b_mn) {
+                    box = 0;
+                    while ((16 << box) < half) ++box;
+                }
+                const CUtensorMap* bmap = box == 3 ? &p.tb : &p.tbs[box];
+                const uint32_t stage_bytes = kQOpBytes + (p.b_mn ? kQOpBytes : (16u << box) * 128u);
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = (int)(it % kQStages);
+                    const uint32_t ph = (it / kQStages) & 1u;
+                    if (!qwait(&empty[s], ph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    uint8_t* st = smem + s * kQStage;
+                    const int k = tl.k0 + kb * kQBK;
+                    const uint32_t fb = full_leader + 8u * s;
                     if (pa) {
-                        mbar_arrive_expect_tx(&full[s], stage_bytes);
-                        load_operand(st, &p.ta, p.a_mn, tl.m0, k, arow, &full[s]);
+                        if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
+                        qload(st, &p.ta, p.a_mn, tl.m0 + 128 * (int)cta, k, arow, fb);
                     } else {
-                        load_operand(st + kBABytes, bhalf ? &p.tb_half : &p.tb, p.b_mn, tl.n0, k, 0,
-                                     &full[s]);
+                        qload(st + kQOpBytes, bmap, p.b_mn, tl.n0 + half * (int)cta, k, 0, fb);
                     }
-                    issued |= 1u << s;
-                    last_ph = (last_ph & ~(1u << s)) | (ph << s);
-                    if (++s == kBStages) { s = 0; ph ^= 1; }
                 }
             }
-            // leave no copy in flight: warp 0 waits for the last fill of every
-            // stage, which counts both producers' copies
-            if (pa)
-                for (int i = 0; i < kBStages; ++i)
-                    if (issued >> i & 1u) wait_bar(&full[i], last_ph >> i & 1u, abort_flag, P.status, true);
+            // The leader's full barriers count both CTAs' copies: its A
+            // producer waits for the last phase of every stage in use.
+            if (leader && pa)
+                for (uint32_t j = it > (uint32_t)kQStages ? it - kQStages : 0u; j < it; ++j)
+                    qwait(&full[j % kQStages], (j / kQStages) & 1u, abort_flag, P.status, true);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (warp == kQMmaWarp) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
             int s = 0, buf = 0;
             uint32_t ph = 0, aph = 0;
             bool ok = true, any = false;
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-                BTile tl;
-                btile_at(P, t, tl);
+            for (int t = pair; ok && t < ntiles; t += npairs) {
+                QTile tl;
+                qtile_at(P, t, tl);
                 const BwdProblem& p = P.p[tl.prob];
-                const int nkb = bk_blocks(tl);
-                // N: the tile's valid columns rounded up to 16 (an M = 128 MMA
-                // takes N in steps of 16), so a ragged row tile pays only for its rows
-                const uint32_t idesc = idesc_bf16_f32_major(kBT, min(kBN, (tl.nvalid + 15) & ~15),
-                                                            p.a_mn, p.b_mn);
-                if (!wait_bar(&tempty[buf], aph ^ 1, abort_flag, P.status)) break;
+                const int nkb = qk_blocks(tl);
+                const uint32_t idesc = idesc_bf16_f32_major(kQM, qtile_n(p, tl), p.a_mn, p.b_mn);
+                if (!qwait(&tempty[buf], aph ^ 1, abort_flag, P.status)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + buf * kBN;
+                const uint32_t d = tmem_base + buf * kQN;
                 bool first = true;
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!wait_bar(&full[s], ph, abort_flag, P.status)) { ok = false; break; }
+                    if (!qwait(&full[s], ph, abort_flag, P.status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t st = smem_addr(smem + s * kBStage);
-                    const int krem = tl.k1 - (tl.k0 + kb * kBBK);  // rows of K left in the range
+                    const uint32_t st = smem_addr(smem + s * kQStage);
+                    const int krem = tl.k1 - (tl.k0 + kb * kQBK);
 #pragma unroll
-                    for (int kk = 0; kk < kBBK / 16; ++kk) {
+                    for (int kk = 0; kk < kQBK / 16; ++kk) {
                         if (16 * kk < krem) {
-                            tc_mma_f16(d, op_desc(st, p.a_mn, kk), op_desc(st + kBABytes, p.b_mn, kk),
-                                       idesc, first ? 0u : 1u);
+                            tc_mma_f16_pair(d, qdesc(st, p.a_mn, kk), qdesc(st + kQOpBytes, p.b_mn, kk),
+                                            idesc, first ? 0u : 1u);
                             first = false;
                         }
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit_pair(&empty[s], 0x3);
                     any = true;
-                    if (++s == kBStages) { s = 0; ph ^= 1; }
+                    if (++s == kQStages) { s = 0; ph ^= 1; }
                 }
                 if (!ok) break;
-                // a tile with an empty K range issues no MMA: the commit then
-                // only orders it after the earlier tiles, and the epilogue
-                // writes zeros without reading tensor memory
-                tc_commit(&tfull[buf]);
+                // a tile with an empty K range issues no MMA; its epilogue writes zeros
+                tc_commit_pair(&tfull[buf], 0x3);
                 any = true;
                 if (++buf == 2) { buf = 0; aph ^= 1; }
             }
             if (any) {
-                tc_commit(mma_done);
-                wait_bar(mma_done, 0, abort_flag, P.status, true);
+                tc_commit_pair(mma_done, 0x1);
+                qwait(mma_done, 0, abort_flag, P.status, true);
             }
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue
-        const int q = warp & 3;           // tensor-memory lane quadrant of this warp
-        const int half = (warp - 2) >> 2;  // columns [64 half, 64 half + 64) of a tile
-        float* stg = epi_smem + (warp - 2) * 32 * 32;
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int hw = (warp - kQEpi0) >> 2;  // columns [128 hw, 128 hw + 128)
+        float* stgs = epi_smem + (warp - kQEpi0) * C::SBUF * 32 * 32;
+        int sb = 0;  // staging tile of the next step
+        const uint32_t tempty_leader = mapa_shared(smem_addr(&tempty[0]), 0);
         int buf = 0;
         uint32_t aph = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-            BTile tl;
-            btile_at(P, t, tl);
+        for (int t = pair; t < ntiles; t += npairs) {
+            QTile tl;
+            qtile_at(P, t, tl);
             const BwdProblem& p = P.p[tl.prob];
-            if (!wait_bar(&tfull[buf], aph, abort_flag, P.status)) break;
+            if (!qwait(&tfull[buf], aph, abort_flag, P.status)) break;
             tc_fence_after();
-            const bool has_k = bk_blocks(tl) > 0;
-            const int m = tl.m0 + q * 32 + lane;
+            const bool has_k = qk_blocks(tl) > 0;
+            const int mrow = tl.m0 + 128 * (int)cta;       // this CTA's first row of D
+            const int m = mrow + q * 32 + lane;
             const bool mok = m < p.M;
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kBN;
-            const int cend = min(tl.nvalid, (kBN / 2) * half + kBN / 2);
-            if (EPI == BEPI_STORE) {
-                const size_t obase = (size_t)tl.grp * (size_t)p.out_grp;
-                const int mq = tl.m0 + q * 32;  // first feature of this warp's 32
-                for (int c0 = (kBN / 2) * half; c0 < cend; c0 += 32) {
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kQN;
+            const int cend = min(tl.nvalid, 128 * hw + 128);
+            if constexpr (EPI == BEPI_STORE) {
+                // staged [rows][32 features] boxes leave in bulk tensor stores
+                // from two alternating staging tiles.  Token-row tiles of a
+                // padded segment store 16-row boxes that start below the
+                // tile's valid rows (a multiple of 16); elsewhere one 32-row
+                // box, which the map clips at the tensor's edge.
+                const int mq = mrow + q * 32;
+                const int g3 = p.rows_as_k ? tl.grp : 0;
+                const bool rows16 = !p.rows_as_k && p.seg != nullptr;
+                for (int c0 = 128 * hw; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);
@@ -331,48 +361,41 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
 #pragma unroll
                         for (int j = 0; j < 32; ++j) r[j] = 0u;
                     }
-                    // transpose: stg[column j][feature lane]
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __uint_as_float(r[j]);
+                    float* stg = stgs + sb * 1024;
+                    uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
+                    if (lane == 0) bulk_wait_read<C::SBUF - 1>();  // this tile's last stores have read it
                     __syncwarp();
                     if (p.out_f32) {
-                        // 8 lanes write one column's 32 features (128 B) as 16-byte chunks
-                        float* out = reinterpret_cast<float*>(p.out) + obase;
 #pragma unroll
-                        for (int it = 0; it < 8; ++it) {
-                            const int row = 4 * it + (lane >> 3), ch = lane & 7;
-                            if (c0 + row < tl.nvalid && mq + 4 * ch < p.M)
-                                *reinterpret_cast<float4*>(out + (size_t)(tl.n0 + c0 + row) * p.ld_out +
-                                                           mq + 4 * ch) =
-                                    *reinterpret_cast<const float4*>(stg + row * 32 + 4 * ch);
-                        }
+                        for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __uint_as_float(r[j]);
                     } else {
-                        // 4 lanes write one column's 32 features (64 B) as 8 bf16 each
-                        uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + obase;
 #pragma unroll
-                        for (int it = 0; it < 4; ++it) {
-                            const int row = 8 * it + (lane >> 2), ch = lane & 3;
-                            if (c0 + row < tl.nvalid && mq + 8 * ch < p.M) {
-                                const float* v = stg + row * 32 + 8 * ch;
-                                uint32_t w4[4];
+                        for (int j = 0; j < 32; ++j) stg16[j * 32 + lane] = qbf(__uint_as_float(r[j]));
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (mq < p.M) {
+                            if (!rows16) {
+                                tma_store_3d(&p.to, stg, mq, tl.n0 + c0, g3);
+                            } else {
 #pragma unroll
-                                for (int h = 0; h < 4; ++h)
-                                    w4[h] = (uint32_t)f2bf(v[2 * h]) | ((uint32_t)f2bf(v[2 * h + 1]) << 16);
-                                *reinterpret_cast<uint4*>(out + (size_t)(tl.n0 + c0 + row) * p.ld_out +
-                                                          mq + 8 * ch) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                                for (int h = 0; h < 2; ++h)
+                                    if (c0 + 16 * h < tl.nvalid)
+                                        tma_store_3d(&p.to,
+                                                     p.out_f32 ? static_cast<const void*>(stg + h * 512)
+                                                               : static_cast<const void*>(stg16 + h * 512),
+                                                     mq, tl.n0 + c0 + 16 * h, g3);
                             }
                         }
+                        bulk_commit();  // one group per step, empty or not
                     }
-                    __syncwarp();
+                    if (++sb == C::SBUF) sb = 0;
                 }
             } else {
-                // SwiGLU backward for 128 features i (lanes) of 32 rows at a
-                // time: with da' = D[i, r] (before the routing weight w),
-                //   a = SiLU(g) u,  da = w da',
-                //   dg = da u sigma(g) (1 + g (1 - sigma(g))),  du = da SiLU(g),
-                // and the routing-weight gradient's partial sum over this
-                // warp's 32 features, sum_i a_i da'_i.
-                for (int c0 = (kBN / 2) * half; c0 < cend; c0 += 32) {
+                // SwiGLU backward (see gemm_bwd.cu): D[i, r] = da'_r[i] for this
+                // CTA's 128 features i, 32 rows at a time
+                for (int c0 = 128 * hw; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
                         tmem_ld_32(tbase + c0, r);
@@ -382,8 +405,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                         for (int j = 0; j < 32; ++j) r[j] = 0u;
                     }
                     float part[32];
-                    // eight rows at a time: their pre-activations and weights are
-                    // loaded (read-only path) before any of the eight rows' stores
 #pragma unroll
                     for (int j0 = 0; j0 < 32; j0 += 8) {
                         float gv[8], uv[8], wv[8];
@@ -408,16 +429,16 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                                 const float da = w * da1;
                                 const float dg = da * u * sg * (1.0f + g * (1.0f - sg));
                                 const float du = da * sl;
-                                p.dgu[(size_t)row * p.ld_dgu + m] = f2bf(dg);
-                                p.dgu[(size_t)row * p.ld_dgu + p.half + m] = f2bf(du);
-                                p.aw[(size_t)row * p.ld_aw + m] = f2bf(w * a);
+                                p.dgu[(size_t)row * p.ld_dgu + m] = qbf(dg);
+                                p.dgu[(size_t)row * p.ld_dgu + p.half + m] = qbf(du);
+                                p.aw[(size_t)row * p.ld_aw + m] = qbf(w * a);
                                 part[j0 + j] = a * da1;
                             }
                         }
                     }
-                    if (p.dw_part) {
-                        // butterfly reduce-scatter over the warp: afterwards lane L
-                        // holds the sum over the 32 lanes of row c0 + L (fixed order)
+                    // a quadrant past the problem's features (M not a multiple of
+                    // 256) writes no partial: I is a multiple of 32
+                    if (p.dw_part && mrow + 32 * q < p.M) {
 #pragma unroll
                         for (int off = 16; off >= 1; off >>= 1) {
                             const bool hi = (lane & off) != 0;
@@ -429,37 +450,51 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_gemm_kernel(const __grid_con
                             }
                         }
                         if (c0 + lane < tl.nvalid)
-                            p.dw_part[(size_t)(tl.n0 + c0 + lane) * p.ld_dw + (tl.m0 >> 5) + q] = part[0];
+                            p.dw_part[(size_t)(tl.n0 + c0 + lane) * p.ld_dw + (mrow >> 5) + q] = part[0];
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) mbar_arrive_cluster(tempty_leader + 8u * buf);
             if (++buf == 2) { buf = 0; aph ^= 1; }
         }
+        if (EPI == BEPI_STORE && lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, kBTmemCols);
+    if (warp == kQMmaWarp) tmem_dealloc_pair(tmem_base, kQTmemCols);
 }
 
 template <int EPI>
-static cudaError_t launch_bwd_t(const BwdParams& params, int grid, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kBSmem);
+static cudaError_t launch_bwd_pair_t(const BwdParams& params, int grid, cudaStream_t s) {
+    constexpr int kQSmem = QCfg<EPI>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(bwd_pair_gemm_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
     if (e != cudaSuccess) return e;
-    bwd_gemm_kernel<EPI><<<grid, kBThreads, kBSmem, s>>>(params);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kQThreads);
+    cfg.dynamicSmemBytes = kQSmem;
+    cfg.stream = s;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, bwd_pair_gemm_kernel<EPI>, &cfg) == cudaSuccess &&
+        clusters > 0 && 2 * clusters < grid)
+        grid = 2 * clusters;
+    cudaGetLastError();
+    bwd_pair_gemm_kernel<EPI><<<grid, kQThreads, kQSmem, s>>>(params);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_gemm(int epi, const BwdParams& params, int grid, cudaStream_t s) {
     if (params.n_problems < 1 || params.n_problems > kBwdMaxProblems) return cudaErrorInvalidValue;
-    if (grid < 1) grid = 1;
-    if (epi == BEPI_STORE) return launch_bwd_t<BEPI_STORE>(params, grid, s);
-    if (epi == BEPI_DSWIGLU) return launch_bwd_t<BEPI_DSWIGLU>(params, grid, s);
+    grid &= ~1;
+    if (grid < 2) grid = 2;
+    if (epi == BEPI_STORE) return launch_bwd_pair_t<BEPI_STORE>(params, grid, s);
+    if (epi == BEPI_DSWIGLU) return launch_bwd_pair_t<BEPI_DSWIGLU>(params, grid, s);
     return cudaErrorInvalidValue;
 }
 

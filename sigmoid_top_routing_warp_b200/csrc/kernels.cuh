@@ -201,10 +201,11 @@ cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cuda
 // ---------------------------------------------------------------- backward GEMMs
 // One problem of a backward grouped GEMM launch (gemm_bwd.cu).  The tensor-
 // memory accumulator of a tile is D[m, n] = sum_k A(m, k) B(n, k) over a
-// 128 x 256 tile, lane = m, column = n; each operand is K-major (a 2-D map
-// [rows, K], box {64, 128} for A and {64, 256} for B) or MN-major (a 3-D view
-// {64, K rows, MN / 64} of the row-major [K, MN] matrix, strides {MN * 2, 128}
-// bytes, box {64, 64, 2} for A and {64, 64, 4} for B).
+// 256 x 256 tile of a CTA pair (128 rows m per CTA, lane = m, column = n);
+// each operand is K-major (a 2-D map [rows, K], box {64, 128}; K-major B also
+// {64, 16 << i}) or MN-major (a 3-D view {64, K rows, MN / 64} of the
+// row-major [K, MN] matrix, strides {MN * 2, 128} bytes, box {64, 64, 2}).
+// Each CTA of the pair stages 128 of the tile's m and half of its n.
 //   rows_as_k = 0: the N dimension runs over token rows, grouped by `seg`
 //     (per group: tiles of 256 rows, prefix `tstart`), K = [0, K); A's row
 //     coordinate is offset by group * a_grp_rows (the group's weights).
@@ -215,12 +216,15 @@ cudaError_t launch_fp8_tm_gemm(int epi, const GemmParams& params, int grid, cuda
 enum BwdEpilogue : int { BEPI_STORE = 0, BEPI_DSWIGLU = 1 };
 struct BwdProblem {
     CUtensorMap ta, tb;
-    CUtensorMap tb_half;      // rows_as_k = 0, K-major B: the same map with a {64, 128} box,
-                              // for row tiles of at most 128 valid rows
+    CUtensorMap tbs[3];       // K-major B: the same operand with boxes {64, 16 << i} rows
+                              // (tb: {64, 128}); MN-major B: tb only, box {64, 64, 2}
+    CUtensorMap to;           // BEPI_STORE: store map of out, 3-D {M, rows, groups}, box
+                              // {32, 16 or 32, 1}
     int a_mn, b_mn;
     int rows_as_k;
     const int32_t* seg;       // [n_grp + 1] group row offsets, or null: one group [0, n_rows)
     const int32_t* tstart;    // rows_as_k = 0 with seg: [n_grp + 1] prefix of 256-row tiles
+    const int32_t* ttab;      // with tstart, or null: [tstart[n_grp]] the group of each row tile
     int n_grp, n_rows;
     int M, N, K;
     int a_grp_rows;
