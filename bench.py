@@ -903,7 +903,7 @@ def backward_object(args, rb, peaks, peak_src, world):
             "ms_per_step": step_ms, "tflops": work["flops"] / (step_ms / 1e3) / 1e12,
             "roofline": {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s",
                          "frac": ach / burst, "traffic": None,
-                         "kernel": "bwd_gemm_kernel (%s)" % dom,
+                         "kernel": "bwd_pair_gemm_kernel (%s)" % dom,
                          "algorithmic_per_launch": work["stages"][dom], "launch_ms": gemm[dom],
                          "peak_kind": "bf16 burst", "peak_source": peak_src,
                          "frac_of_sustained_peak":
