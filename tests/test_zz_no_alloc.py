@@ -37,7 +37,7 @@ def routing(T, E, k, seed, skew=False):
 
 def permute_both(B, cfg, idx):
     dev = "cuda"
-    n = cfg.T * cfg.k
+    n = max(cfg.T * cfg.k, 1)  # the entry points take non-NULL rows / pos even when T = 0
     ref = [torch.full((cfg.E + 1,), -7, dtype=torch.int32, device=dev),
            torch.full((n,), -7, dtype=torch.int32, device=dev),
            torch.full((n,), -7, dtype=torch.int32, device=dev)]
