@@ -419,6 +419,24 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const void* w_
                           float* dw13s, float* dw2s, float* dlogits, void* ws, size_t ws_bytes,
                           void* const* stage_events, moe_stream_t stream);
 
+/* Expert-bias update of noaux_tc routing (the training side of the selection
+ * bias).  mlqm.cn 稀疏激活 names noaux_tc (a per-expert bias steers the
+ * top-k choice and stays out of the routing weights; no auxiliary loss) but
+ * prints no update rule; the rule here is the plainest reading of it: after
+ * a routed batch, each expert whose load is above the batch mean loses gamma
+ * from its bias, each one below gains gamma, one exactly at the mean keeps it:
+ *   load_e = #{(t, j) : topk_idx[t, j] = e},   b_e += gamma * sign(T*k/E - load_e)
+ * The comparison is exact (integers); the update is one fp32 addition.
+ *   topk_idx int32 [T, k]   the batch's choice (moe_route); entries outside
+ *                           [0, E) count for no expert
+ *   bias     fp32 [E]       in/out, updated in place
+ *   gamma    >= 0, finite   the step
+ * One launch (one block; its histogram is integer, so the result does not
+ * depend on scheduling).  T = 0 leaves the bias unchanged and launches
+ * nothing.  Returns MOE_ERR_INVALID_ARG for NULL pointers or a bad gamma.   */
+moe_status_t moe_bias_update(const moe_config_t* cfg, const int32_t* topk_idx, float* bias,
+                             float gamma, moe_stream_t stream);
+
 /* Synchronise `stream`, read the workspace status block of `ws` (the layer's
  * or the DSA indexer's) and clear it.  Returns MOE_OK; MOE_ERR_TIMEOUT if a
  * kernel gave up a bounded wait; or MOE_ERR_WORKSPACE if a tile-claim counter

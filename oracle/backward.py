@@ -20,7 +20,8 @@ out step by step below:
   out = sum_j w_j y_j + shared(x)
 
 The expert bias b gets no gradient (noaux_tc balances load with a separate
-update rule, which the pages do not give).
+update rule, which the pages do not print; balance.py holds the reading of
+it that the library implements).
 """
 from __future__ import annotations
 

@@ -35,8 +35,8 @@ WS_ITEMS = {"logits": 0, "topk_idx": 1, "topk_w": 2, "offsets": 3, "rows": 4, "p
 
 # Every symbol include/moe.h declares.
 EXPORTED = ("moe_get_last_error", "moe_workspace_size", "moe_workspace_offset", "moe_route",
-            "moe_route_from_logits", "moe_permute", "moe_expert_ffn", "moe_combine",
-            "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
+            "moe_route_from_logits", "moe_bias_update", "moe_permute", "moe_expert_ffn",
+            "moe_combine", "moe_forward", "moe_check_device_status", "moe_permute_noalloc",
             "moe_quantize_act", "moe_rmsnorm", "moe_forward_block",
             "moe_backward_workspace_size", "moe_backward", "moe_ep_pack",
             "moe_shared_expert", "moe_ep_expert_counts", "moe_ep_plan", "moe_ep_dispatch_peer",
@@ -99,6 +99,8 @@ _lib.moe_route.restype = ctypes.c_int
 _lib.moe_route.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_route_from_logits.restype = ctypes.c_int
 _lib.moe_route_from_logits.argtypes = [_CFG, _P, _P, _P, _P, _P]
+_lib.moe_bias_update.restype = ctypes.c_int
+_lib.moe_bias_update.argtypes = [_CFG, _P, _P, ctypes.c_float, _P]
 _lib.moe_permute.restype = ctypes.c_int
 _lib.moe_permute.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_expert_ffn.restype = ctypes.c_int
@@ -217,6 +219,14 @@ def moe_route_from_logits(cfg, logits, bias, topk_idx, topk_w, stream=None):
     c = cfg.c()
     _check(_lib.moe_route_from_logits(ctypes.byref(c), _ptr(logits), _ptr(bias), _ptr(topk_idx),
                                       _ptr(topk_w), _stream(stream)), "moe_route_from_logits")
+
+
+def moe_bias_update(cfg, topk_idx, bias, gamma, stream=None):
+    """noaux_tc expert-bias update in place: bias[e] += gamma * sign(mean load
+    - load_e) over the batch's choices topk_idx [T, k]."""
+    c = cfg.c()
+    _check(_lib.moe_bias_update(ctypes.byref(c), _ptr(topk_idx), _ptr(bias), float(gamma),
+                                _stream(stream)), "moe_bias_update")
 
 
 def moe_permute(cfg, topk_idx, offsets, rows, pos, ws, stream=None):

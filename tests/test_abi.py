@@ -97,6 +97,23 @@ def test_calls_reject_bad_arguments_before_launch(B):
     assert st == B.MOE_ERR_INVALID_ARG
 
 
+def test_bias_update_rejects_bad_arguments_before_launch(B):
+    L = B.lib()
+    cc = cfg(B).c()
+    for g in (float("nan"), -1.0, float("inf")):
+        st = L.moe_bias_update(ctypes.byref(cc), None, None, g, None)
+        assert st == B.MOE_ERR_INVALID_ARG and "gamma" in B.get_last_error()
+    st = L.moe_bias_update(ctypes.byref(cc), None, 16, 1e-3, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "topk_idx" in B.get_last_error()
+    st = L.moe_bias_update(ctypes.byref(cc), 16, None, 1e-3, None)
+    assert st == B.MOE_ERR_INVALID_ARG and "bias" in B.get_last_error()
+    bad = cfg(B, E=33).c()
+    assert L.moe_bias_update(ctypes.byref(bad), 16, 16, 1e-3, None) != B.MOE_OK
+    # T = 0: nothing to count, nothing launched
+    empty = cfg(B, T=0).c()
+    assert L.moe_bias_update(ctypes.byref(empty), 16, 16, 1e-3, None) == B.MOE_OK
+
+
 def test_empty_batch_is_a_no_op(B):
     c = cfg(B, T=0)
     cc = c.c()
