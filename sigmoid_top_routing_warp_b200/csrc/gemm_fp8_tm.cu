@@ -19,13 +19,16 @@
 // which suits a few tokens per expert but makes the scale vary along the
 // accumulator's columns.)
 //
-// Roles (18 warps): warp 0 issues TMA loads (operands per K block; the
+// Roles (10 warps): warp 0 issues TMA loads (operands per K block; the
 // scales of four K blocks at a time into a small ring: s_x for the tile's
 // 128 rows as one {4, 128} box, s_w as two {4, 1} boxes), warp 1 allocates
-// tensor memory and issues the MMAs (one thread), warps 2-17 promote and
-// finish: warp w reads TMEM lane quadrant w % 4 and column group (w - 2) / 4.
-// Two 256-column partial buffers let the MMAs of block kb+1 run while block
-// kb is promoted.
+// tensor memory and issues the MMAs (one thread), warps 2-9 promote and
+// finish: warp w reads TMEM lane quadrant w % 4 and column group (w - 2) / 4,
+// 128 of the 256 columns, into 128 fp32 register accumulators (with 320
+// threads, three warps on a sub-partition, a thread may hold 168 registers).
+// Each K block is promoted in sixteen 8-column chunks whose TMEM loads run
+// one chunk ahead of the FMAs.  Two 256-column partial buffers let the MMAs
+// of block kb+1 run while block kb is promoted.
 //
 // EPI_SWIGLU: a = SiLU(gate) * up, quantised per token over the tile's 128
 // features (one e4m3 block of A); the four column groups exchange their
@@ -59,10 +62,10 @@ constexpr int kTMStages = 4;
 constexpr int kTMGroup = 4;                    // K blocks per scale fetch
 constexpr int kTMSSlots = 3;                   // scale ring depth
 constexpr int kTMSSlot = 2304;                 // s_x [128][4] at 0, s_w rows at 2048 and 2176
-constexpr int kTMEpiWarps = 16;
+constexpr int kTMEpiWarps = 8;
 constexpr int kTMThreads = 64 + 32 * kTMEpiWarps;
 constexpr int kTMNP = 2;                       // partial buffers of kTMN columns
-constexpr int kTMAmaxBytes = 2 * 4 * kTMTok * 4;  // [2 parities][4 column groups][128 rows]
+constexpr int kTMAmaxBytes = 2 * 2 * kTMTok * 4;  // [2 parities][2 column groups][128 rows]
 constexpr int kTMBarBytes = 512;
 constexpr int kTMRing = 4;                     // claimed tile ids in flight (producer -> MMA, epilogue)
 constexpr int kTMSchedWord = 24;               // first scheduling word in the status block
@@ -281,14 +284,14 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     } else {
         // ------------------------------------------------ epilogue: promote, then finish the tile
         const int q = warp & 3;              // TMEM lane quadrant: rows 32q .. 32q + 31
-        const int g = (warp - 2) >> 2;       // column group
+        const int g = (warp - 2) >> 2;       // column group 0 or 1
         const int tok = 32 * q + lane;       // this thread's row of the tile
-        // accumulator columns: SWIGLU gate [32g, 32g+32) and up [128+32g, ...);
-        // SCALE [64g, 64g+64), both halves in weight-scale block g / 2
-        const uint32_t ca = EPI == EPI_SWIGLU ? 32 * g : 64 * g;
-        const uint32_t cb = EPI == EPI_SWIGLU ? 128 + 32 * g : 64 * g + 32;
-        const int swa = EPI == EPI_SWIGLU ? 0 : (g >> 1);
-        const int swb = EPI == EPI_SWIGLU ? 1 : (g >> 1);
+        // accumulator columns: SWIGLU gate [64g, 64g+64) and up [128+64g, ...);
+        // SCALE [128g, 128g+128), all in weight-scale block g
+        const uint32_t ca = EPI == EPI_SWIGLU ? 64 * g : 128 * g;
+        const uint32_t cb = EPI == EPI_SWIGLU ? 128 + 64 * g : 128 * g + 64;
+        const int swa = EPI == EPI_SWIGLU ? 0 : g;
+        const int swb = EPI == EPI_SWIGLU ? 1 : g;
         int pb = 0, ss = 0, tile_no = 0;
         uint32_t pph = 0, sph = 0;
         bool ok = true;
@@ -307,9 +310,9 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             const int nk = p.K / kTMBK;
             const bool valid = tok < tl.nvalid;
             const int row = tl.row0 + tok;
-            float acc[64];
+            float acc[128];
 #pragma unroll
-            for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
             for (int kb0 = 0; kb0 < nk && ok; kb0 += kTMGroup) {
                 if (!wait_bar(&sfull[ss], sph, abort_flag, P.status)) { ok = false; break; }
                 const float* sl = reinterpret_cast<const float*>(sring + ss * kTMSSlot);
@@ -322,19 +325,31 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                     if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + pb * kTMN;
-                    tm_promote16(tb + ca, sa, acc);
-                    tm_promote16(tb + ca + 16, sa, acc + 16);
-                    tm_promote16(tb + cb, sb, acc + 32);
-                    // the last 16 columns: the partial is released as soon as they
-                    // are in registers, before their FMAs
-                    uint32_t r[16];
-                    tmem_ld_16(tb + cb + 16, r);
+                    // sixteen 8-column chunks (eight at ca, eight at cb); chunk c + 1
+                    // is loaded while chunk c is accumulated, and the partial is
+                    // released once the last chunk is in registers
+                    uint32_t r[2][8];
+                    tmem_ld_8(tb + ca, r[0]);
                     tmem_wait_ld();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pempty[pb]);
 #pragma unroll
-                    for (int j = 0; j < 16; j += 2) tm_ffma2(acc[48 + j], acc[49 + j], sb, r[j], r[j + 1]);
+                    for (int c = 0; c < 16; ++c) {
+                        if (c + 1 < 16) {
+                            const uint32_t col = c + 1 < 8 ? ca + 8 * (c + 1) : cb + 8 * (c - 7);
+                            tmem_ld_8(tb + col, r[(c + 1) & 1]);
+                        }
+                        const uint64_t sc2 = c < 8 ? sa : sb;
+#pragma unroll
+                        for (int j = 0; j < 8; j += 2)
+                            tm_ffma2(acc[8 * c + j], acc[8 * c + j + 1], sc2, r[c & 1][j], r[c & 1][j + 1]);
+                        if (c + 1 < 16) {
+                            tmem_wait_ld();
+                            if (c + 1 == 15) {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&pempty[pb]);
+                            }
+                        }
+                    }
                     if (++pb == kTMNP) { pb = 0; pph ^= 1; }
                 }
                 __syncwarp();
@@ -343,55 +358,58 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             }
             if (!ok) break;
             if (EPI == EPI_SWIGLU) {
-                // a = SiLU(gate) * up for features f0 + 32g .. + 31 of this row
+                // a = SiLU(gate) * up for features f0 + 64g .. + 63 of this row
                 float m = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    acc[j] = silu_q(acc[j]) * acc[32 + j];
+                for (int j = 0; j < 64; ++j) {
+                    acc[j] = silu_q(acc[j]) * acc[64 + j];
                     m = fmaxf(m, fabsf(acc[j]));
                 }
                 const int par = tile_no & 1;
-                amax_sm[(par * 4 + g) * kTMTok + tok] = m;
+                amax_sm[(par * 2 + g) * kTMTok + tok] = m;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&amax_bar[par]);
                 if (!wait_bar(&amax_bar[par], (tile_no >> 1) & 1, abort_flag, P.status)) break;
-                const float* all = amax_sm + par * 4 * kTMTok + tok;
-                const float amax = fmaxf(fmaxf(all[0], all[kTMTok]), fmaxf(all[2 * kTMTok], all[3 * kTMTok]));
+                const float* all = amax_sm + par * 2 * kTMTok + tok;
+                const float amax = fmaxf(all[0], all[kTMTok]);
                 const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
                 // codes: a * (1 / sc), the reciprocal rounded once (within one fp32
                 // ulp of a / sc before the e4m3 rounding), two per conversion
                 const float inv = __frcp_rn(sc);
                 if (valid) {
-                    uint32_t packed[8];
+                    uint4* dst = reinterpret_cast<uint4*>(p.out_q + (size_t)row * p.ld_out + tl.f0 + 64 * g);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-                            make_float2(acc[4 * w] * inv, acc[4 * w + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-                        const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-                            make_float2(acc[4 * w + 2] * inv, acc[4 * w + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-                        packed[w] = lo | (hi << 16);
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t packed[4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const int j = 16 * v + 4 * w;
+                            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                                make_float2(acc[j] * inv, acc[j + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+                            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                                make_float2(acc[j + 2] * inv, acc[j + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+                            packed[w] = lo | (hi << 16);
+                        }
+                        dst[v] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(p.out_q + (size_t)row * p.ld_out + tl.f0 + 32 * g);
-                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                     if (g == 0) p.out_scale[(size_t)row * (p.ld_out / 128) + tl.f0 / 128] = sc;
                 }
             } else {
-                const int f = tl.f0 + 64 * g;
+                const int f = tl.f0 + 128 * g;
                 if (valid && f < p.n_feat) {
                     const float wr = p.row_w ? __ldg(p.row_w + row) : 1.0f;
                     if (p.out_f32) {
                         float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
                                                                 (size_t)row * p.ld_out + f);
 #pragma unroll
-                        for (int v = 0; v < 16; ++v)
+                        for (int v = 0; v < 32; ++v)
                             dst[v] = make_float4(acc[4 * v] * wr, acc[4 * v + 1] * wr,
                                                  acc[4 * v + 2] * wr, acc[4 * v + 3] * wr);
                     } else {
                         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
                                                               (size_t)row * p.ld_out + f);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
+                        for (int v = 0; v < 16; ++v) {
                             uint32_t w4[4];
 #pragma unroll
                             for (int h = 0; h < 4; ++h) {
