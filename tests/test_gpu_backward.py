@@ -131,6 +131,8 @@ CASES = [
     ("grouped_no_shared", 200, 512, 64, 6, 128, 0, 4, 2, True, 1.0, "uniform"),
     ("k1", 150, 512, 32, 1, 128, 1, 1, 1, True, 1.0, "uniform"),
     ("one_token", 1, 512, 32, 8, 256, 1, 1, 1, True, 1.0, "uniform"),
+    # M = I = 384 and H = 768 end half-way into a 256-row pair tile; group routing
+    ("half_pair_tiles", 333, 768, 64, 6, 384, 2, 8, 4, True, 1.0, "uniform"),
 ]
 
 
