@@ -225,7 +225,17 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a, int gat
         if (row < 0) continue;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)(s / a.k) * a.H);
         uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)row * a.H);
-        for (int c = lane; c < chunks; c += 32) dst[c] = __ldg(src + c);
+        // four chunks per lane in flight before their stores
+        int c = lane;
+        for (; c + 96 < chunks; c += 128) {
+            const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32), v2 = __ldg(src + c + 64),
+                        v3 = __ldg(src + c + 96);
+            dst[c] = v0;
+            dst[c + 32] = v1;
+            dst[c + 64] = v2;
+            dst[c + 96] = v3;
+        }
+        for (; c < chunks; c += 32) dst[c] = __ldg(src + c);
         if (lane == 0) a.w_perm[row] = a.topk_w[s];
     }
 }
@@ -249,25 +259,40 @@ __global__ void __launch_bounds__(64) combine_kernel(const CombineArgs a) {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < a.k; ++j) {
-        const int r = a.pos[(size_t)t * a.k + j];
-        if (r < 0) continue;
-        if (a.y_f32) {
+    if (a.y_f32) {
+        for (int j = 0; j < a.k; ++j) {
+            const int r = a.pos[(size_t)t * a.k + j];
+            if (r < 0) continue;
             const float4* yr = reinterpret_cast<const float4*>(
                                    static_cast<const float*>(a.y) + (size_t)r * a.H) + 2 * c;
             const float4 v0 = __ldg(yr), v1 = __ldg(yr + 1);
             acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
             acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
-            continue;
         }
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                                  static_cast<const uint16_t*>(a.y) + (size_t)r * a.H) + c);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+    } else {
+        // eight slots at a time: their rows' loads are all issued before the
+        // sums, which still run in slot order
+        for (int j0 = 0; j0 < a.k; j0 += 8) {
+            int r[8];
+            uint4 v[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(p[i]);
-            acc[2 * i] += f.x;
-            acc[2 * i + 1] += f.y;
+            for (int i = 0; i < 8; ++i) r[i] = j0 + i < a.k ? __ldg(a.pos + (size_t)t * a.k + j0 + i) : -1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (r[i] >= 0)
+                    v[i] = __ldg(reinterpret_cast<const uint4*>(
+                                     static_cast<const uint16_t*>(a.y) + (size_t)r[i] * a.H) + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (r[i] < 0) continue;
+                const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f = __bfloat1622float2(p[h]);
+                    acc[2 * h] += f.x;
+                    acc[2 * h + 1] += f.y;
+                }
+            }
         }
     }
     if (a.y_shared) {
