@@ -217,3 +217,26 @@ def test_peer_plan_flags_a_receive_buffer_too_small(B, W):
     assert (sb.cpu().numpy() == 5).all()
     assert (ro.cpu().numpy() == np.arange(el + 1) * 10).all()
     assert (ident.cpu().numpy() == np.arange(100)).all()
+
+
+@pytest.mark.parametrize("form", ["all_to_all", "peer"])
+def test_every_choice_on_one_rank(B, W, form):
+    """A bias that puts every token's choice among rank 0's experts: the other
+    ranks own experts nobody chose and receive no rows (empty exchanges and
+    empty expert segments on three of four ranks); every rank's output still
+    equals moe_forward's bit for bit."""
+    from sigmoid_top_routing_warp_b200 import ep
+    wl = W.Workload("ep_skew", T=80, H=512, E=128, k=4, I=128, n_shared=1, seed=29)
+    inp = W.make_inputs(wl, device="cuda")
+    N = 4
+    bias = torch.full((wl.E,), -20.0, device="cuda")
+    bias[: wl.E // N] = 20.0  # rank 0's 32 experts win every choice
+    inp = dict(inp, bias=bias)
+    xs = tokens_of(W, wl, N, wl.T, seed=77)
+    cfg = mk_cfg(B, wl, wl.T)
+    run = ep.ep_forward_peer_virtual if form == "peer" else ep.ep_forward_virtual
+    outs = run(cfg, xs, inp["w_router"], inp["bias"], inp["w13"], inp["w2"], inp["w13s"], inp["w2s"])
+    torch.cuda.synchronize()
+    for r in range(N):
+        check_rank(B, cfg, inp, xs[r], outs[r], "%s skewed rank %d" % (form, r),
+                   tokens=[0, wl.T // 2, wl.T - 1])
