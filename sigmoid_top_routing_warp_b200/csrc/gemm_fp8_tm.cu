@@ -26,8 +26,8 @@
 // finish: warp w reads TMEM lane quadrant w % 4 and column group (w - 2) / 4,
 // 128 of the 256 columns, into 128 fp32 register accumulators (with 320
 // threads, three warps on a sub-partition, a thread may hold 168 registers).
-// Each K block is promoted in sixteen 8-column chunks whose TMEM loads run
-// one chunk ahead of the FMAs.  Two 256-column partial buffers let the MMAs
+// Each K block is promoted in 8-column (gate/up) or 16-column (down) chunks
+// whose TMEM loads run one chunk ahead of the FMAs.  Two 256-column partial buffers let the MMAs
 // of block kb+1 run while block kb is promoted.
 //
 // EPI_SWIGLU: a = SiLU(gate) * up, quantised per token over the tile's 128
@@ -110,13 +110,13 @@ __device__ __forceinline__ void tm_ffma2(float& a0, float& a1, uint64_t ss, uint
 // one; 0 for a gate below about -88, where exp overflows).
 __device__ __forceinline__ float silu_q(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// Promote 16 columns of a partial: acc[j] += s * P[j].
-__device__ __forceinline__ void tm_promote16(uint32_t taddr, uint64_t ss, float* acc) {
-    uint32_t r[16];
-    tmem_ld_16(taddr, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < 16; j += 2) tm_ffma2(acc[j], acc[j + 1], ss, r[j], r[j + 1]);
+// A chunk of CH (8 or 16) tensor-memory columns of this thread's lane.
+template <int CH>
+__device__ __forceinline__ void tm_ld_chunk(uint32_t taddr, uint32_t (&r)[CH]) {
+    if constexpr (CH == 16)
+        tmem_ld_16(taddr, r);
+    else
+        tmem_ld_8(taddr, r);
 }
 
 }  // namespace
@@ -325,25 +325,30 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                     if (!wait_bar(&pfull[pb], pph, abort_flag, P.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + pb * kTMN;
-                    // sixteen 8-column chunks (eight at ca, eight at cb); chunk c + 1
-                    // is loaded while chunk c is accumulated, and the partial is
-                    // released once the last chunk is in registers
-                    uint32_t r[2][8];
-                    tmem_ld_8(tb + ca, r[0]);
+                    // NCH chunks of CH columns (half at ca, half at cb): 8-column
+                    // chunks for the gate/up GEMM, 16 for the down GEMM (measured
+                    // best for each); chunk c + 1 is loaded while chunk c is
+                    // accumulated, and the partial is released once the last chunk
+                    // is in registers
+                    constexpr int CH = EPI == EPI_SWIGLU ? 8 : 16;
+                    constexpr int NCH = 128 / CH;
+                    uint32_t r[2][CH];
+                    tm_ld_chunk<CH>(tb + ca, r[0]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (c + 1 < 16) {
-                            const uint32_t col = c + 1 < 8 ? ca + 8 * (c + 1) : cb + 8 * (c - 7);
-                            tmem_ld_8(tb + col, r[(c + 1) & 1]);
+                    for (int c = 0; c < NCH; ++c) {
+                        if (c + 1 < NCH) {
+                            const int c1 = c + 1;
+                            const uint32_t col = c1 < NCH / 2 ? ca + CH * c1 : cb + CH * (c1 - NCH / 2);
+                            tm_ld_chunk<CH>(tb + col, r[c1 & 1]);
                         }
-                        const uint64_t sc2 = c < 8 ? sa : sb;
+                        const uint64_t sc2 = c < NCH / 2 ? sa : sb;
 #pragma unroll
-                        for (int j = 0; j < 8; j += 2)
-                            tm_ffma2(acc[8 * c + j], acc[8 * c + j + 1], sc2, r[c & 1][j], r[c & 1][j + 1]);
-                        if (c + 1 < 16) {
+                        for (int j = 0; j < CH; j += 2)
+                            tm_ffma2(acc[CH * c + j], acc[CH * c + j + 1], sc2, r[c & 1][j], r[c & 1][j + 1]);
+                        if (c + 1 < NCH) {
                             tmem_wait_ld();
-                            if (c + 1 == 15) {
+                            if (c + 1 == NCH - 1) {
                                 tc_fence_before();
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(&pempty[pb]);
