@@ -15,7 +15,8 @@
 // epilogue writes its 128 rows.
 //
 // N per tile: token rows (K-major B) use the tile's valid rows rounded up to
-// 16, each CTA supplying half of them; output columns (MN-major B) use 256.
+// 16, each CTA supplying half of them from the smallest of its 16-, 32-, 64-
+// or 128-row boxes that holds them; output columns (MN-major B) use 256.
 //
 // Roles per CTA (352 threads): warp 0 loads A and (leader) sets the stage's
 // expected bytes for both CTAs, warp 1 loads B, warp 2 holds the tensor
@@ -393,8 +394,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kQThreads, 1)
                     if (++sb == C::SBUF) sb = 0;
                 }
             } else {
-                // SwiGLU backward (see gemm_bwd.cu): D[i, r] = da'_r[i] for this
-                // CTA's 128 features i, 32 rows at a time
+                // SwiGLU backward: D[i, r] = da'_r[i] (the row's output gradient
+                // times W2's column i, before the routing weight w_r) for this
+                // CTA's 128 features i, 32 rows at a time.  With s = sigmoid(g),
+                // a = SiLU(g) u and da = w_r da':
+                //   dg = da u s (1 + g (1 - s)),  du = da SiLU(g),
+                // stored bf16 with w_r a (the down weights' gradient operand);
+                // the routing weight's gradient sum_i a_i da'_i goes out as
+                // per-warp partials over 32 features
                 for (int c0 = 128 * hw; c0 < cend; c0 += 32) {
                     uint32_t r[32];
                     if (has_k) {
