@@ -90,7 +90,7 @@ class OracleSteps:
         return out
 
 
-def _rank(rank, world, port, q):
+def _rank(rank, world, port, q, skew=False):
     os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
                       MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
@@ -104,6 +104,10 @@ def _rank(rank, world, port, q):
     try:
         wl = W.Workload("ep_tiny", T=40, H=128, E=32, k=4, I=128, n_shared=1, seed=0)
         inp = W.make_inputs(wl, device="cpu")  # the same weights on every rank
+        if skew:  # every choice among rank 0's experts: rank 1 receives no rows
+            bias = torch.full((wl.E,), -20.0)
+            bias[: wl.E // world] = 20.0
+            inp = dict(inp, bias=bias)
         g = torch.Generator().manual_seed(100 + rank)
         x = (torch.randn((wl.T, wl.H), generator=g)).to(torch.bfloat16)  # this rank's tokens
         cfg = MoeConfig(T=wl.T, H=wl.H, E=wl.E, k=wl.k, I=wl.I, n_shared=1)
@@ -126,17 +130,28 @@ def _rank(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_expert_parallel_protocol_two_ranks_gloo():
+def run_two_ranks(skew):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q, skew)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=300)
     assert all(p.exitcode == 0 for p in procs)
-    got = sorted(q.get(timeout=5) for _ in range(2))
-    for rank, err, owners in got:
+    return sorted(q.get(timeout=5) for _ in range(2))
+
+
+def test_expert_parallel_protocol_two_ranks_gloo():
+    for rank, err, owners in run_two_ranks(skew=False):
         assert err < 1e-12, (rank, err)
         assert owners == [0, 1], (rank, owners)
+
+
+def test_expert_parallel_protocol_empty_exchanges_gloo():
+    """Every choice on rank 0's experts: rank 1 sends all its rows to rank 0,
+    rank 0 sends none, and rank 1 runs its expert step on zero rows."""
+    for rank, err, owners in run_two_ranks(skew=True):
+        assert err < 1e-12, (rank, err)
+        assert owners == [0], (rank, owners)
