@@ -49,6 +49,10 @@ constexpr uint32_t kQChunk = kQBK * 128;           // one 64-wide MN chunk: 64 K
 constexpr int kQBarBytes = 256;
 constexpr int kQTmemCols = 2 * kQN;
 constexpr long long kQWaitLimit = 1ll << 31;
+// the launch passes every problem's tensor maps by value (4.75 KB for
+// five problems): within the 32,764-byte kernel parameter limit of sm_70+
+// with CUDA 12.1 and later
+static_assert(sizeof(BwdParams) <= 32764, "kernel parameter size");
 // Shared memory per epilogue: stores keep five operand stages and two 4 KB
 // staging tiles per epilogue warp; the SwiGLU backward needs no staging and
 // takes six stages.
