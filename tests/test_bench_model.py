@@ -32,3 +32,37 @@ def test_gate_up_share_of_the_stream():
     w1 = bench.layer_work(d, touched=1)["g1_bytes"]
     w2 = bench.layer_work(d, touched=2)["g1_bytes"]
     assert w2 - w1 == 2 * 5120 * 1536 * 2
+
+
+def test_traffic_record_selection(tmp_path, monkeypatch):
+    """profile_traffic: a record counts only while its source hash matches;
+    an exact-workload byte count beats a ratio taken on this workload's
+    shape, which beats a generic ratio for the kernel."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "a.md").write_text(
+        "text\n\n    kernel: k1\n    traffic_over_algorithmic: 1.50\n    source_hash: old\n\n"
+        "    kernel: k1\n    traffic_over_algorithmic: 1.10\n    source_hash: cur\n")
+    (prof / "b.md").write_text(
+        "    kernel: k1\n    workload: w2\n    traffic_over_algorithmic: 1.20\n    source_hash: cur\n"
+        "\n    kernel: k1\n    workload: w3\n    traffic_bytes_per_launch: 777\n    source_hash: cur\n"
+        "\n    kernel: k2\n    traffic_over_algorithmic: 9.0\n    source_hash: cur\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_hash", lambda kind: "cur")
+    assert abs(bench.profile_traffic("k1", 100.0, "w1") - 110.0) < 1e-9   # generic ratio
+    assert abs(bench.profile_traffic("k1", 100.0, "w2") - 120.0) < 1e-9   # this shape's ratio
+    assert bench.profile_traffic("k1", 100.0, "w3") == 777.0               # measured bytes
+    assert bench.profile_traffic("k3", 100.0, "w1") is None                # no record
+    monkeypatch.setattr(bench, "source_hash", lambda kind: "new")
+    assert bench.profile_traffic("k1", 100.0, "w1") is None                # kernel changed
+
+
+def test_committed_traffic_records_name_known_kernels():
+    # every machine-read record under profiles/ names a kernel kind the bench knows
+    import os
+    import re
+    kinds = set(bench.KERNEL_SOURCES)
+    for name in os.listdir(os.path.join(bench.ROOT, "profiles")):
+        text = open(os.path.join(bench.ROOT, "profiles", name)).read()
+        for k in re.findall(r"^    kernel: (\S+)$", text, flags=re.M):
+            assert k in kinds, (name, k)
